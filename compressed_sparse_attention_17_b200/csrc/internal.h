@@ -1,0 +1,54 @@
+// internal.h - launchers shared between the C-ABI layer and the kernels.
+// Host-side declarations only; arguments are validated by the caller.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+// Device address of the library error word on the current device.
+int* device_error_ptr();
+
+// Counts one kernel launch (csa_kernel_launches()).
+void count_launches(int n = 1);
+
+// ---- SIMT kernels (simt.cu): every dtype, every shape the ABI accepts ----
+cudaError_t launch_rmsnorm_rope(const csa_geom& g, int in_dt, int out_dt, const void* x,
+                                int64_t rows, const int64_t* pos, int64_t pos0, int64_t pos_step,
+                                const float* gain, void* out, const int64_t* out_row,
+                                cudaStream_t s);
+cudaError_t launch_quantize_mixed(int in_dt, const void* x, int64_t rows, void* out,
+                                  cudaStream_t s);
+// P[T, nW*c] (FP32) = H[T,d] @ [W_0 | ... | W_{nW-1}], each W_i [d, c].
+cudaError_t launch_proj_simt(int dt, const void* H, int64_t T, int d, int c, int nW,
+                             const void* const* W, float* P, cudaStream_t s);
+// Pool + RMSNorm + RoPE of every complete block from projections P.
+cudaError_t launch_pool_prefill(const csa_geom& g, const float* P, int64_t T, const float* bias,
+                                const float* gain, int out_dt, void* E, cudaStream_t s);
+cudaError_t launch_decode_proj(const csa_geom& g, int dt, const void* h, const int64_t* pos,
+                               int B, int d, const void* const* W, int nW, float* state,
+                               cudaStream_t s);
+cudaError_t launch_decode_pool(const csa_geom& g, const int64_t* pos, int B, const float* bias,
+                               const float* gain, const float* state, int out_dt, void* E,
+                               int64_t ldE, cudaStream_t s);
+cudaError_t launch_index_scores_simt(const csa_geom& g, int dt, const void* qI, const float* w,
+                                     const void* KI, int64_t ldK, const int32_t* seq_of_q,
+                                     const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
+                                     int c_I, float* scores, int64_t ld_scores, cudaStream_t s);
+cudaError_t launch_topk_from_scores(const csa_geom& g, const float* scores, int64_t ld_scores,
+                                    const int32_t* seq_of_q, const int64_t* pos,
+                                    const int64_t* n_entries, int Q, int k, int32_t* idx_out,
+                                    float* scores_dbg, int64_t ld_dbg, cudaStream_t s);
+// dense != 0: HCA (all visible entries); else CSA with idx [Q, k].
+cudaError_t launch_attend_simt(const csa_geom& g, int q_dt, int kv_dt, const void* q,
+                               const float* q_gain, const float* sink, const void* E,
+                               int64_t ldE, const int64_t* n_entries, const int32_t* idx, int k,
+                               int dense, const void* win, int64_t ldW, const int32_t* seq_of_q,
+                               const int64_t* pos, int Q, int H_q, void* O, cudaStream_t s);
+bool attend_simt_supported(int c, int H_q);
+
+}  // namespace csa

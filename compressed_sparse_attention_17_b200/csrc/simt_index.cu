@@ -1,0 +1,234 @@
+// simt_index.cu - CUDA-core lightning-indexer scores and radix top-k.
+//
+// These kernels accept every dtype and shape the C ABI accepts. They are the
+// FP32 path (FP32 arithmetic throughout, as the FP32 workloads require) and
+// the path for shapes the tensor-core kernels do not cover.
+//
+// Equations: "Evidence Ledger" CSA Eqs 9-19, HCA Eqs 20-26, Shared attention
+// details (Sec 2.3.3, Eq 27); "DeepSeek-V4" study 03 (pooling and index-score
+// formulas).
+#include <cfloat>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace csa {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Index scores on CUDA cores: I[q,s] = sum_h w[q,h] ReLU(qI[q,h] . KI[s]).
+// Block = 128 entries of one query; KI tile staged in shared memory with a
+// padded row stride; each thread accumulates its entry's H_I head dots.
+// ---------------------------------------------------------------------------
+template <typename Tin, int HMAX>
+__global__ void __launch_bounds__(128) index_scores_simt_kernel(
+    csa_geom g, const Tin* __restrict__ qI, const float* __restrict__ w,
+    const Tin* __restrict__ KI, int64_t ldK, const int32_t* __restrict__ seq_of_q,
+    const int64_t* __restrict__ pos, const int64_t* __restrict__ n_entries, int H_I, int c_I,
+    float* __restrict__ scores, int64_t ld_scores) {
+  extern __shared__ float smem[];
+  const int q = blockIdx.y;
+  const int b = seq_of_q[q];
+  const int64_t nv = n_visible(pos[q], g.m, g.vis_offset, min(n_entries[b], ldK));
+  const int64_t s0 = (int64_t)blockIdx.x * 128;
+  if (s0 >= nv) return;
+  float* qs = smem;                   // [H_I][c_I]
+  float* ws = qs + H_I * c_I;         // [H_I]
+  float* ks = ws + HMAX;              // [128][c_I + 1]
+  for (int e = threadIdx.x; e < H_I * c_I; e += 128) qs[e] = to_f32(qI[(int64_t)q * H_I * c_I + e]);
+  for (int e = threadIdx.x; e < H_I; e += 128) ws[e] = w[(int64_t)q * H_I + e];
+  const int ld = c_I + 1;
+  const Tin* kb = KI + ((int64_t)b * ldK + s0) * c_I;
+  for (int e = threadIdx.x; e < 128 * c_I; e += 128) {
+    int rr = e / c_I, j = e % c_I;
+    ks[rr * ld + j] = (s0 + rr < nv) ? to_f32(kb[(int64_t)rr * c_I + j]) : 0.f;
+  }
+  __syncthreads();
+  const int64_t s = s0 + threadIdx.x;
+  if (s >= nv) return;
+  float acc[HMAX];
+#pragma unroll
+  for (int h = 0; h < HMAX; ++h) acc[h] = 0.f;
+  const float* kr = ks + threadIdx.x * ld;
+  for (int j = 0; j < c_I; ++j) {
+    const float kv = kr[j];
+#pragma unroll
+    for (int h = 0; h < HMAX; ++h)
+      if (h < H_I) acc[h] = fmaf(qs[h * c_I + j], kv, acc[h]);
+  }
+  float I = 0.f;
+#pragma unroll
+  for (int h = 0; h < HMAX; ++h)
+    if (h < H_I) I = fmaf(ws[h], fmaxf(acc[h], 0.f), I);
+  scores[(int64_t)q * ld_scores + s] = I;
+}
+
+// ---------------------------------------------------------------------------
+// Top-k by radix select on order-preserving 32-bit keys, one block per
+// query; ties at the threshold keep the lowest indices; output ascending.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kTopkThreads = 1024;
+
+template <int NT>
+__device__ int block_exclusive_scan(int v, int* sh, int* total) {
+  // sh: NT/32 ints scratch
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int s = lane < NT / 32 ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < NT / 32) sh[lane] = s;
+  }
+  __syncthreads();
+  int base = wid > 0 ? sh[wid - 1] : 0;
+  *total = sh[NT / 32 - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(
+    csa_geom g, const float* __restrict__ scores, int64_t ld_scores,
+    const int32_t* __restrict__ seq_of_q, const int64_t* __restrict__ pos,
+    const int64_t* __restrict__ n_entries, int k, int32_t* __restrict__ idx_out,
+    float* __restrict__ scores_dbg, int64_t ld_dbg) {
+  __shared__ int hist[256];
+  __shared__ int scan_sh[kTopkThreads / 32];
+  __shared__ uint32_t sh_prefix;
+  __shared__ int sh_remaining;
+  const int q = blockIdx.x;
+  const int b = seq_of_q[q];
+  const int64_t nv = n_visible(pos[q], g.m, g.vis_offset, min(n_entries[b], ld_scores));
+  const float* sc = scores + (int64_t)q * ld_scores;
+  int32_t* out = idx_out + (int64_t)q * k;
+  if (scores_dbg)
+    for (int64_t s = threadIdx.x; s < nv; s += kTopkThreads) scores_dbg[(int64_t)q * ld_dbg + s] = sc[s];
+  if (nv <= k) {
+    for (int64_t j = threadIdx.x; j < k; j += kTopkThreads) out[j] = j < nv ? (int32_t)j : -1;
+    return;
+  }
+  // radix select of the k-th largest key, 8 bits per pass from the top
+  uint32_t prefix = 0, mask = 0;
+  int remaining = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int e = threadIdx.x; e < 256; e += kTopkThreads) hist[e] = 0;
+    __syncthreads();
+    for (int64_t s = threadIdx.x; s < nv; s += kTopkThreads) {
+      uint32_t key = order_key(sc[s]);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int cum = 0, dsel = 0;
+      for (int dg = 255; dg >= 0; --dg) {
+        if (cum + hist[dg] >= remaining) {
+          dsel = dg;
+          break;
+        }
+        cum += hist[dg];
+      }
+      sh_prefix = prefix | ((uint32_t)dsel << shift);
+      sh_remaining = remaining - cum;
+    }
+    __syncthreads();
+    prefix = sh_prefix;
+    remaining = sh_remaining;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  // prefix = threshold key; `remaining` ties at the threshold are kept
+  const uint32_t thr = prefix;
+  const int64_t per = (nv + kTopkThreads - 1) / kTopkThreads;
+  const int64_t a0 = threadIdx.x * per;
+  const int64_t a1 = min(nv, a0 + per);
+  int nsel = 0, ntie = 0;
+  for (int64_t s = a0; s < a1; ++s) {
+    uint32_t key = order_key(sc[s]);
+    nsel += key > thr;
+    ntie += key == thr;
+  }
+  int tot;
+  const int tie_base = block_exclusive_scan<kTopkThreads>(ntie, scan_sh, &tot);
+  int take_ties = remaining - tie_base;
+  take_ties = take_ties < 0 ? 0 : (take_ties > ntie ? ntie : take_ties);
+  const int out_base = block_exclusive_scan<kTopkThreads>(nsel + take_ties, scan_sh, &tot);
+  int o = out_base, tl = 0;
+  for (int64_t s = a0; s < a1; ++s) {
+    uint32_t key = order_key(sc[s]);
+    bool keep = key > thr;
+    if (key == thr) {
+      keep = tl < take_ties;
+      ++tl;
+    }
+    if (keep) out[o++] = (int32_t)s;
+  }
+  // k_eff = k here (nv > k)
+}
+
+}  // namespace
+
+template <typename Tin, int HMAX>
+static cudaError_t index_simt_t(const csa_geom& g, const void* qI, const float* w, const void* KI,
+                                int64_t ldK, const int32_t* seq_of_q, const int64_t* pos,
+                                const int64_t* n_entries, int Q, int H_I, int c_I, float* scores,
+                                int64_t ld_scores, cudaStream_t s) {
+  size_t smem = sizeof(float) * ((size_t)H_I * c_I + HMAX + 128 * (size_t)(c_I + 1));
+  auto kern = index_scores_simt_kernel<Tin, HMAX>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((ldK + 127) / 128), (unsigned)Q);
+  count_launches();
+  kern<<<grid, 128, smem, s>>>(g, reinterpret_cast<const Tin*>(qI), w,
+                               reinterpret_cast<const Tin*>(KI), ldK, seq_of_q, pos, n_entries,
+                               H_I, c_I, scores, ld_scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_index_scores_simt(const csa_geom& g, int dt, const void* qI, const float* w,
+                                     const void* KI, int64_t ldK, const int32_t* seq_of_q,
+                                     const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
+                                     int c_I, float* scores, int64_t ld_scores, cudaStream_t s) {
+  if (Q == 0 || ldK == 0) return cudaSuccess;
+#define CSA_IDX_CASE(HM)                                                                       \
+  if (H_I <= HM)                                                                               \
+    return dt == CSA_F32                                                                       \
+               ? index_simt_t<float, HM>(g, qI, w, KI, ldK, seq_of_q, pos, n_entries, Q, H_I,  \
+                                         c_I, scores, ld_scores, s)                            \
+               : index_simt_t<__nv_bfloat16, HM>(g, qI, w, KI, ldK, seq_of_q, pos, n_entries,  \
+                                                 Q, H_I, c_I, scores, ld_scores, s);
+  CSA_IDX_CASE(8)
+  CSA_IDX_CASE(32)
+  CSA_IDX_CASE(64)
+  CSA_IDX_CASE(128)
+#undef CSA_IDX_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_topk_from_scores(const csa_geom& g, const float* scores, int64_t ld_scores,
+                                    const int32_t* seq_of_q, const int64_t* pos,
+                                    const int64_t* n_entries, int Q, int k, int32_t* idx_out,
+                                    float* scores_dbg, int64_t ld_dbg, cudaStream_t s) {
+  if (Q == 0) return cudaSuccess;
+  count_launches();
+  topk_kernel<<<Q, kTopkThreads, 0, s>>>(g, scores, ld_scores, seq_of_q, pos, n_entries, k,
+                                         idx_out, scores_dbg, ld_dbg);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -15,7 +15,9 @@ tensors. Any subset of rows can thus be regenerated without drawing the rest.
 from __future__ import annotations
 
 import math
+import os
 import zlib
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -65,13 +67,24 @@ class Spec:
             v = bf16_bits_to_f32(f32_to_bf16_bits(v))
         return v
 
+    def _fill(self, out: np.ndarray, convert) -> np.ndarray:
+        n = self.nrows
+        nchunks = math.ceil(n / CHUNK_ROWS)
+
+        def one(j):
+            out[j * CHUNK_ROWS:(j + 1) * CHUNK_ROWS] = convert(self._chunk(j))
+
+        if nchunks > 4:
+            with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+                list(ex.map(one, range(nchunks)))
+        else:
+            for j in range(nchunks):
+                one(j)
+        return out.reshape(self.shape)
+
     def values(self) -> np.ndarray:
         """All values as float32 (exactly representable in the storage type)."""
-        n = self.nrows
-        out = np.empty((n, self.width), np.float32)
-        for j in range(math.ceil(n / CHUNK_ROWS)):
-            out[j * CHUNK_ROWS:(j + 1) * CHUNK_ROWS] = self._chunk(j)
-        return out.reshape(self.shape)
+        return self._fill(np.empty((self.nrows, self.width), np.float32), lambda v: v)
 
     def rows(self, flat_rows) -> np.ndarray:
         """Values of the given flat row indices (rows of the last dim)."""
@@ -85,8 +98,10 @@ class Spec:
 
     def storage(self) -> np.ndarray:
         """Stored representation: uint16 BF16 bits or float32 values."""
-        v = self.values()
-        return f32_to_bf16_bits(v) if self.dtype == "bf16" else v
+        if self.dtype == "bf16":
+            return self._fill(np.empty((self.nrows, self.width), np.uint16),
+                              lambda v: (v.view(np.uint32) >> 16).astype(np.uint16))
+        return self.values()
 
 
 # ---------------------------------------------------------------------------

@@ -90,7 +90,7 @@ typedef enum {
 typedef struct {
   int m;            /* tokens per compressed entry: 4 (CSA) or 128 (HCA) */
   int overlap;      /* 1: CSA, 2m candidates per entry; 0: HCA, m candidates */
-  int c;            /* entry width = attention head width; multiple of 64 */
+  int c;            /* entry width = attention head width; multiple of 16, <= 1024 */
   int rope_dims;    /* RoPE on the last rope_dims dims; even, <= c */
   double rope_base; /* RoPE base, 10000 */
   float eps;        /* RMSNorm epsilon, 1e-6 */
@@ -106,6 +106,10 @@ const char* csa_status_string(csa_status s);
 /* Library version string (static). */
 const char* csa_version(void);
 
+/* Number of CUDA kernels this library has launched in the process so far
+ * (all devices, all streams). Lets a caller count the library's work. */
+uint64_t csa_kernel_launches(void);
+
 /* Synchronises `stream`, then reads and clears the device error word that
  * bounded device-side waits set. Returns CSA_ERR_TIMEOUT if a wait gave up
  * since the last call, CSA_ERR_CUDA on a CUDA error, else CSA_OK. */
@@ -120,14 +124,16 @@ csa_status csa_sync_status(csa_stream_t stream);
  * pos0 + r * pos_step.
  *   x    [rows, c] in_dtype (F32 or BF16)
  *   gain [c] FP32, NULL = all ones
- *   out  [rows, c] out_dtype (F32, BF16), or [rows] mixed rows of
+ *   out  output rows of width c, out_dtype (F32, BF16), or mixed rows of
  *        CSA_MIXED_ROW_BYTES when out_dtype = CSA_FP8_MIXED (c = 512,
- *        rope_dims = 64 only).
+ *        rope_dims = 64 only). Row r is written to output row out_row[r]
+ *        when `out_row` (device int64 [rows]) is non-NULL - e.g. slot
+ *        b*n_win + (p mod n_win) of a decode window ring - else to row r.
  * --------------------------------------------------------------------- */
 csa_status csa_rmsnorm_rope(const csa_geom* g, csa_dtype in_dtype, csa_dtype out_dtype,
                             const void* x, int64_t rows, const int64_t* pos, int64_t pos0,
                             int64_t pos_step, const float* gain, void* out,
-                            csa_stream_t stream);
+                            const int64_t* out_row, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------
  * csa_quantize_mixed - store rows of width 512 in the CSA_FP8_MIXED layout
@@ -204,7 +210,8 @@ csa_status csa_compress_decode(const csa_geom* g, csa_dtype dtype, const void* h
  *   idx_out   [Q, k] int32
  *   scores_dbg [Q, ldK] FP32 or NULL: when given, the kernel's FP32 scores
  *             for s < n_vis(q) (other slots untouched) - a diagnostic.
- * 1 <= k <= CSA_MAX_TOPK; c_I multiple of 16; H_I <= 128.
+ * 1 <= k <= CSA_MAX_TOPK; c_I a multiple of 16, <= 256; H_I <= 128.
+ * n_vis is also clipped to ldK.
  * workspace: csa_index_topk_workspace_size() bytes.
  * --------------------------------------------------------------------- */
 size_t csa_index_topk_workspace_size(int Q, int64_t ldK, int k);
@@ -229,7 +236,8 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
  *   q     [Q, H_q, c] q_dtype (F32 or BF16); O [Q, H_q, c] q_dtype
  *   q_gain [c] FP32 or NULL (ones); sink [H_q] FP32
  *   E     [nseq, ldE, c] kv_dtype (F32, BF16, or mixed rows)
- *   idx   [Q, k] int32, entries < n_entries[b] or -1
+ *   idx   [Q, k] int32, entries < n_entries[b] or -1 (slots holding -1 or
+ *         an index >= ldE are skipped)
  *   win   [nseq, ldW, c] kv_dtype (F32 or BF16), rows already prepared
  *         (csa_rmsnorm_rope); row of position j = j (win_ring = 0, ldW > p)
  *         or j mod n_win (win_ring = 1, ldW >= n_win).
