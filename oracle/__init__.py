@@ -90,7 +90,7 @@ def rmsnorm(x, eps=1e-6, gain=None):
     x = _f64(x)
     c = x.shape[-1]
     y = np.empty_like(x)
-    g = _f64(gain)
+    g = _f64(gain)  # kept referenced until the call returns
     lib.orc_rmsnorm_rows(_ptr(x), x.size // c, c, _ptr(g), eps, _ptr(y))
     return y
 
@@ -112,8 +112,8 @@ def rmsnorm_rope(x, pos, rope_dims, base=10000.0, eps=1e-6, gain=None):
     rows = x.size // c
     p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, dtype=np.float64), x.shape[:-1]))
     y = np.empty_like(x)
-    lib.orc_rmsnorm_rope_rows(_ptr(x), rows, c, rope_dims, base, eps, _ptr(_f64(gain)), _ptr(p),
-                              _ptr(y))
+    g = _f64(gain)
+    lib.orc_rmsnorm_rope_rows(_ptr(x), rows, c, rope_dims, base, eps, _ptr(g), _ptr(p), _ptr(y))
     return y
 
 
@@ -161,7 +161,8 @@ def index_topk(qI, w, KI, seq_of_q, pos, n_entries, m, k, vis_offset=1, want_sco
     tau = np.empty(Q, np.float64)
     amag = np.empty(Q, np.float64)
     scores = np.full((Q, ldK), np.nan) if want_scores else None
-    rc = lib.orc_index_topk(Q, HI, cI, k, m, vis_offset, _ptr(qI), _ptr(_f64(w)), _ptr(KI), ldK,
+    w = _f64(w)
+    rc = lib.orc_index_topk(Q, HI, cI, k, m, vis_offset, _ptr(qI), _ptr(w), _ptr(KI), ldK,
                             _ptr(seq), _ptr(pos), _ptr(ne), _ptr(idx), _ptr(tau), _ptr(amag),
                             _ptr(scores))
     if rc != 0:
@@ -187,8 +188,9 @@ def attend(q, sink, E, win, seq_of_q, pos, n_entries, *, rope_dims, idx=None, m=
     k = 0 if idx is None else idxa.shape[1]
     O = np.empty_like(q)
     nk = np.empty(Q, np.int32)
+    qg, sk = _f64(q_gain), _f64(sink)
     rc = lib.orc_attend(Q, Hq, c, rope_dims, base, eps, n_win, win_ring, _ptr(q),
-                        _ptr(_f64(q_gain)), _ptr(_f64(sink)), _ptr(E), E.shape[1], _ptr(ne),
+                        _ptr(qg), _ptr(sk), _ptr(E), E.shape[1], _ptr(ne),
                         _ptr(idxa), k, dense, m, vis_offset, _ptr(win), win.shape[1], _ptr(seq),
                         _ptr(pos), _ptr(O), _ptr(nk))
     if rc != 0:

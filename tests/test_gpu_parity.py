@@ -228,7 +228,7 @@ def test_index_topk_no_visible_entries(orc):
 
 
 # ------------------------------------------------------------------ attention
-def _attend_case(Q, Hq, c, r, nseq, N, k, dt, kv="same", ring=False, seed=7, hole=0.1):
+def _attend_case(orc, Q, Hq, c, r, nseq, N, k, dt, kv="same", ring=False, seed=7, hole=0.1):
     rg = np.random.default_rng(seed)
     q = _spec("q", (Q, Hq, c), 1.0, dt, seed).values()
     E = _spec("E", (nseq, N, c), 1.0, "bf16" if kv == "mixed" else dt, seed).values()
@@ -249,7 +249,7 @@ def _attend_case(Q, Hq, c, r, nseq, N, k, dt, kv="same", ring=False, seed=7, hol
                                                ("bf16", 64, 512, 64, 96, True),
                                                ("bf16", 16, 256, 64, 40, False)])
 def test_csa_attend(orc, dt, Hq, c, r, k, ring):
-    q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(13, Hq, c, r, 3, 300, k, dt, ring=ring)
+    q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(orc, 13, Hq, c, r, 3, 300, k, dt, ring=ring)
     g = csa.geom(c=c, rope_dims=r, win_ring=int(ring))
     O = csa.attend(dev(q, dt), dev(sink, "f32"), dev(E, dt), dev_i(idx, torch.int32), dev(win, dt),
                    dev_i(seq, torch.int32), dev_i(pos), dev_i(ne), g, q_gain=dev(gain, "f32"))
@@ -261,7 +261,7 @@ def test_csa_attend(orc, dt, Hq, c, r, k, ring):
 @pytest.mark.parametrize("dt,m", [("bf16", 128), ("f32", 4)])
 def test_hca_attend(orc, dt, m):
     Q, Hq, c, r, N = 11, 8, 256, 64, 40
-    q, E, win, sink, gain, seq, ne, pos, _ = _attend_case(Q, Hq, c, r, 2, N, 8, dt)
+    q, E, win, sink, gain, seq, ne, pos, _ = _attend_case(orc, Q, Hq, c, r, 2, N, 8, dt)
     pos = np.random.default_rng(9).integers(0, m * N + 50, Q).astype(np.int64)
     pos[0] = 0
     ldW = win.shape[1]
@@ -275,7 +275,7 @@ def test_hca_attend(orc, dt, m):
 
 def test_csa_attend_mixed_entries(orc):
     Q, Hq, c, r, N, k = 9, 64, 512, 64, 200, 64
-    q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(Q, Hq, c, r, 2, N, k, "bf16",
+    q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(orc, Q, Hq, c, r, 2, N, k, "bf16",
                                                             kv="mixed", ring=True)
     rows_gpu = csa.quantize_mixed(dev(E.reshape(-1, 512), "bf16")).reshape(2, N, -1)
     rows_orc = orc.pack_mixed(E.reshape(-1, 512)).reshape(2, N, -1)
