@@ -64,14 +64,14 @@ _SIGS = {
     "csa_compress_decode": ([_GP, _I32, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P,
                              _I64, _P], _I32),
     "csa_index_topk_workspace_size": ([_I32, _I64, _I32], _SZ),
-    "csa_index_topk": ([_GP, _I32, _P, _P, _P, _I64, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P,
-                        _P, _SZ, _P], _I32),
+    "csa_index_topk": ([_GP, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _I32, _I32, _I32,
+                        _P, _P, _P, _SZ, _P], _I32),
     "csa_attend_workspace_size": ([_I32, _I32, _I32, _I32, _I32], _SZ),
-    "csa_attend": ([_GP, _I32, _I32, _P, _P, _P, _P, _I64, _P, _P, _I32, _P, _I64, _P, _P, _I32,
-                    _I32, _P, _P, _SZ, _P], _I32),
+    "csa_attend": ([_GP, _I32, _I32, _P, _P, _P, _P, _I64, _I32, _P, _P, _I32, _P, _I64, _P, _P,
+                    _I32, _I32, _P, _P, _SZ, _P], _I32),
     "hca_attend_workspace_size": ([_I32, _I32, _I32, _I64, _I32], _SZ),
-    "hca_attend": ([_GP, _I32, _I32, _P, _P, _P, _P, _I64, _P, _P, _I64, _P, _P, _I32, _I32, _P,
-                    _P, _SZ, _P], _I32),
+    "hca_attend": ([_GP, _I32, _I32, _P, _P, _P, _P, _I64, _I32, _P, _P, _I64, _P, _P, _I32, _I32,
+                    _P, _P, _SZ, _P], _I32),
 }
 
 
@@ -211,7 +211,7 @@ def index_topk(qI, w, KI, seq_of_q, pos, n_entries, k, g: Geom, want_scores=Fals
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=qI.device)
     _call("csa_index_topk", ctypes.byref(g), _dt(qI), _ptr(qI), _ptr(w), _ptr(KI), ldK,
-          _ptr(seq_of_q), _ptr(pos), _ptr(n_entries), Q, HI, cI, k, _ptr(idx), _ptr(scores),
+          KI.shape[0], _ptr(seq_of_q), _ptr(pos), _ptr(n_entries), Q, HI, cI, k, _ptr(idx), _ptr(scores),
           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(qI))
     return (idx, scores) if want_scores else idx
 
@@ -227,7 +227,7 @@ def attend(q, sink, E, idx, win, seq_of_q, pos, n_entries, g: Geom, q_gain=None,
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     _call("csa_attend", ctypes.byref(g), _dt(q), _dt(E), _ptr(q), _ptr(q_gain), _ptr(sink),
-          _ptr(E), E.shape[1], _ptr(n_entries), _ptr(idx), k, _ptr(win), win.shape[1],
+          _ptr(E), E.shape[1], E.shape[0], _ptr(n_entries), _ptr(idx), k, _ptr(win), win.shape[1],
           _ptr(seq_of_q), _ptr(pos), Q, Hq, _ptr(O), _ptr(workspace),
           0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(q))
     return O
@@ -243,7 +243,7 @@ def hca_attend(q, sink, E, win, seq_of_q, pos, n_entries, g: Geom, q_gain=None, 
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     _call("hca_attend", ctypes.byref(g), _dt(q), _dt(E), _ptr(q), _ptr(q_gain), _ptr(sink),
-          _ptr(E), E.shape[1], _ptr(n_entries), _ptr(win), win.shape[1], _ptr(seq_of_q),
+          _ptr(E), E.shape[1], E.shape[0], _ptr(n_entries), _ptr(win), win.shape[1], _ptr(seq_of_q),
           _ptr(pos), Q, Hq, _ptr(O), _ptr(workspace),
           0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(q))
     return O

@@ -173,13 +173,13 @@ size_t csa_index_topk_workspace_size(int Q, int64_t ldK, int k) {
 }
 
 csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, const float* w,
-                          const void* KI, int64_t ldK, const int32_t* seq_of_q,
+                          const void* KI, int64_t ldK, int nseq, const int32_t* seq_of_q,
                           const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
                           int c_I, int k, int32_t* idx_out, float* scores_dbg,
                           void* workspace, size_t ws_bytes, csa_stream_t stream) {
   if (!geom_ok(g) || !io_dtype_ok(dtype)) return CSA_ERR_INVALID_ARG;
   if (Q < 0 || H_I < 1 || H_I > 128 || c_I < 16 || (c_I % 16) != 0 || c_I > 256) return CSA_ERR_INVALID_ARG;
-  if (k < 1 || k > CSA_MAX_TOPK || ldK < 0) return CSA_ERR_INVALID_ARG;
+  if (k < 1 || k > CSA_MAX_TOPK || ldK < 0 || nseq < 0) return CSA_ERR_INVALID_ARG;
   if (Q == 0) return CSA_OK;
   if (!qI || !w || !KI || !seq_of_q || !pos || !n_entries || !idx_out) return CSA_ERR_INVALID_ARG;
   const void* ptrs[] = {qI, w, KI, seq_of_q, pos, n_entries, idx_out, scores_dbg, workspace};
@@ -189,13 +189,17 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
     return CSA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* scores = reinterpret_cast<float*>(workspace);
-  if (ldK > 0) {
-    cudaError_t e = csa::launch_index_scores_simt(*g, dtype, qI, w, KI, ldK, seq_of_q, pos,
-                                                  n_entries, Q, H_I, c_I, scores, ldK, s);
+  if (ldK > 0 && nseq > 0) {
+    cudaError_t e = csa::index_tc_supported(dtype, H_I, c_I)
+                        ? csa::launch_index_scores_tc(*g, qI, w, KI, ldK, nseq, seq_of_q, pos,
+                                                      n_entries, Q, H_I, c_I, scores, ldK, s)
+                        : csa::launch_index_scores_simt(*g, dtype, qI, w, KI, ldK, nseq, seq_of_q,
+                                                        pos, n_entries, Q, H_I, c_I, scores, ldK,
+                                                        s);
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
-  return cuda_status(csa::launch_topk_from_scores(*g, scores, ldK, seq_of_q, pos, n_entries, Q, k,
-                                                  idx_out, scores_dbg, ldK, s));
+  return cuda_status(csa::launch_topk_from_scores(*g, scores, ldK, nseq, seq_of_q, pos, n_entries,
+                                                  Q, k, idx_out, scores_dbg, ldK, s));
 }
 
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win) {
@@ -205,13 +209,13 @@ size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win) {
 
 static csa_status attend_common(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype,
                                 const void* q, const float* q_gain, const float* sink,
-                                const void* E, int64_t ldE, const int64_t* n_entries,
+                                const void* E, int64_t ldE, int nseq, const int64_t* n_entries,
                                 const int32_t* idx, int k, int dense, const void* win,
                                 int64_t ldW, const int32_t* seq_of_q, const int64_t* pos, int Q,
                                 int H_q, void* O, csa_stream_t stream) {
   if (!geom_ok(g) || !io_dtype_ok(q_dtype)) return CSA_ERR_INVALID_ARG;
   if (!(io_dtype_ok(kv_dtype) || (kv_dtype == CSA_FP8_MIXED && mixed_ok(g)))) return CSA_ERR_INVALID_ARG;
-  if (Q < 0 || H_q < 1 || ldE < 0 || ldW < 0) return CSA_ERR_INVALID_ARG;
+  if (Q < 0 || H_q < 1 || ldE < 0 || ldW < 0 || nseq < 0) return CSA_ERR_INVALID_ARG;
   if (!dense && (k < 0 || k > CSA_MAX_TOPK)) return CSA_ERR_INVALID_ARG;
   if (Q == 0) return CSA_OK;
   if (!q || !sink || !seq_of_q || !pos || !O || !n_entries) return CSA_ERR_INVALID_ARG;
@@ -222,19 +226,21 @@ static csa_status attend_common(const csa_geom* g, csa_dtype q_dtype, csa_dtype 
   for (const void* p : ptrs)
     if (!aligned16(p)) return CSA_ERR_INVALID_ARG;
   if (!csa::attend_simt_supported(g->c, H_q)) return CSA_ERR_UNSUPPORTED;
-  return cuda_status(launch_attend_simt(*g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, n_entries,
-                                        idx, k, dense, win, ldW, seq_of_q, pos, Q, H_q, O,
+  return cuda_status(launch_attend_simt(*g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, nseq,
+                                        n_entries, idx, k, dense, win, ldW, seq_of_q, pos, Q, H_q, O,
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
 csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,
                       const float* q_gain, const float* sink, const void* E, int64_t ldE,
-                      const int64_t* n_entries, const int32_t* idx, int k, const void* win,
-                      int64_t ldW, const int32_t* seq_of_q, const int64_t* pos, int Q, int H_q,
-                      void* O, void* workspace, size_t ws_bytes, csa_stream_t stream) {
+                      int nseq, const int64_t* n_entries, const int32_t* idx, int k,
+                      const void* win, int64_t ldW, const int32_t* seq_of_q, const int64_t* pos,
+                      int Q, int H_q, void* O, void* workspace, size_t ws_bytes,
+                      csa_stream_t stream) {
   (void)workspace;
   (void)ws_bytes;
-  return attend_common(g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, n_entries, idx, k, 0, win,
+  return attend_common(g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, nseq, n_entries, idx, k, 0,
+                       win,
                        ldW, seq_of_q, pos, Q, H_q, O, stream);
 }
 
@@ -245,12 +251,13 @@ size_t hca_attend_workspace_size(int Q, int H_q, int c, int64_t ldE, int n_win) 
 
 csa_status hca_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,
                       const float* q_gain, const float* sink, const void* E, int64_t ldE,
-                      const int64_t* n_entries, const void* win, int64_t ldW,
+                      int nseq, const int64_t* n_entries, const void* win, int64_t ldW,
                       const int32_t* seq_of_q, const int64_t* pos, int Q, int H_q, void* O,
                       void* workspace, size_t ws_bytes, csa_stream_t stream) {
   (void)workspace;
   (void)ws_bytes;
-  return attend_common(g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, n_entries, nullptr, 0, 1,
+  return attend_common(g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, nseq, n_entries, nullptr, 0,
+                       1,
                        win, ldW, seq_of_q, pos, Q, H_q, O, stream);
 }
 

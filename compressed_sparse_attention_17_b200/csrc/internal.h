@@ -36,17 +36,26 @@ cudaError_t launch_decode_pool(const csa_geom& g, const int64_t* pos, int B, con
                                const float* gain, const float* state, int out_dt, void* E,
                                int64_t ldE, cudaStream_t s);
 cudaError_t launch_index_scores_simt(const csa_geom& g, int dt, const void* qI, const float* w,
-                                     const void* KI, int64_t ldK, const int32_t* seq_of_q,
+                                     const void* KI, int64_t ldK, int nseq,
+                                     const int32_t* seq_of_q,
                                      const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
                                      int c_I, float* scores, int64_t ld_scores, cudaStream_t s);
 cudaError_t launch_topk_from_scores(const csa_geom& g, const float* scores, int64_t ld_scores,
-                                    const int32_t* seq_of_q, const int64_t* pos,
+                                    int nseq, const int32_t* seq_of_q, const int64_t* pos,
                                     const int64_t* n_entries, int Q, int k, int32_t* idx_out,
                                     float* scores_dbg, int64_t ld_dbg, cudaStream_t s);
+// ---- tensor-core kernels (tc_*.cu) ----
+bool index_tc_supported(int dt, int H_I, int c_I);
+cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const float* w,
+                                   const void* KI, int64_t ldK, int nseq,
+                                   const int32_t* seq_of_q, const int64_t* pos,
+                                   const int64_t* n_entries, int Q, int H_I, int c_I,
+                                   float* scores, int64_t ld_scores, cudaStream_t s);
 // dense != 0: HCA (all visible entries); else CSA with idx [Q, k].
 cudaError_t launch_attend_simt(const csa_geom& g, int q_dt, int kv_dt, const void* q,
                                const float* q_gain, const float* sink, const void* E,
-                               int64_t ldE, const int64_t* n_entries, const int32_t* idx, int k,
+                               int64_t ldE, int nseq, const int64_t* n_entries,
+                               const int32_t* idx, int k,
                                int dense, const void* win, int64_t ldW, const int32_t* seq_of_q,
                                const int64_t* pos, int Q, int H_q, void* O, cudaStream_t s);
 bool attend_simt_supported(int c, int H_q);

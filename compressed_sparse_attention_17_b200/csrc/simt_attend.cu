@@ -43,7 +43,7 @@ __device__ __forceinline__ const void* key_row(const csa_geom& g, int kv_dt, con
 template <typename Tq, int OPT>
 __global__ void __launch_bounds__(kAttThreads) attend_simt_kernel(
     csa_geom g, int kv_dt, const Tq* __restrict__ q, const float* __restrict__ q_gain,
-    const float* __restrict__ sink, const void* __restrict__ E, int64_t ldE,
+    const float* __restrict__ sink, const void* __restrict__ E, int64_t ldE, int nseq,
     const int64_t* __restrict__ n_entries, const int32_t* __restrict__ idx, int k, int dense,
     const void* __restrict__ win, int64_t ldW, const int32_t* __restrict__ seq_of_q,
     const int64_t* __restrict__ pos, int H_q, Tq* __restrict__ O) {
@@ -59,6 +59,11 @@ __global__ void __launch_bounds__(kAttThreads) attend_simt_kernel(
   const int qi = blockIdx.x;
   const int b = seq_of_q[qi];
   const int64_t p = pos[qi];
+  if (b < 0 || b >= nseq) {  // no such sequence: zero output
+    for (int e = threadIdx.x; e < H_q * c; e += kAttThreads)
+      O[(int64_t)qi * H_q * c + e] = from_f32<Tq>(0.f);
+    return;
+  }
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int nwarps = kAttThreads / 32;
   // q-hat = RoPE_p(RMSNorm(q_h) * q_gain), one warp per head
@@ -211,7 +216,7 @@ bool attend_simt_supported(int c, int H_q) {
 
 template <typename Tq, int OPT>
 static cudaError_t attend_t(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,
-                            const float* sink, const void* E, int64_t ldE,
+                            const float* sink, const void* E, int64_t ldE, int nseq,
                             const int64_t* n_entries, const int32_t* idx, int k, int dense,
                             const void* win, int64_t ldW, const int32_t* seq_of_q,
                             const int64_t* pos, int Q, int H_q, void* O, cudaStream_t s) {
@@ -221,25 +226,26 @@ static cudaError_t attend_t(const csa_geom& g, int kv_dt, const void* q, const f
   if (e != cudaSuccess) return e;
   count_launches();
   kern<<<Q, kAttThreads, smem, s>>>(g, kv_dt, reinterpret_cast<const Tq*>(q), q_gain, sink, E,
-                                    ldE, n_entries, idx, k, dense, win, ldW, seq_of_q, pos, H_q,
+                                    ldE, nseq, n_entries, idx, k, dense, win, ldW, seq_of_q, pos, H_q,
                                     reinterpret_cast<Tq*>(O));
   return cudaGetLastError();
 }
 
 cudaError_t launch_attend_simt(const csa_geom& g, int q_dt, int kv_dt, const void* q,
                                const float* q_gain, const float* sink, const void* E,
-                               int64_t ldE, const int64_t* n_entries, const int32_t* idx, int k,
+                               int64_t ldE, int nseq, const int64_t* n_entries,
+                               const int32_t* idx, int k,
                                int dense, const void* win, int64_t ldW, const int32_t* seq_of_q,
                                const int64_t* pos, int Q, int H_q, void* O, cudaStream_t s) {
   if (Q == 0) return cudaSuccess;
   const int opt = attend_opt(g.c, H_q);
 #define CSA_ATT_CASE(OP)                                                                        \
   if (opt == OP)                                                                                \
-    return q_dt == CSA_F32 ? attend_t<float, OP>(g, kv_dt, q, q_gain, sink, E, ldE, n_entries,  \
+    return q_dt == CSA_F32 ? attend_t<float, OP>(g, kv_dt, q, q_gain, sink, E, ldE, nseq, n_entries,  \
                                                  idx, k, dense, win, ldW, seq_of_q, pos, Q,     \
                                                  H_q, O, s)                                     \
                            : attend_t<__nv_bfloat16, OP>(g, kv_dt, q, q_gain, sink, E, ldE,     \
-                                                         n_entries, idx, k, dense, win, ldW,    \
+                                                         nseq, n_entries, idx, k, dense, win, ldW,    \
                                                          seq_of_q, pos, Q, H_q, O, s);
   CSA_ATT_CASE(2)
   CSA_ATT_CASE(4)

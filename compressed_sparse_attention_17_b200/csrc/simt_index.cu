@@ -24,12 +24,13 @@ namespace {
 template <typename Tin, int HMAX>
 __global__ void __launch_bounds__(128) index_scores_simt_kernel(
     csa_geom g, const Tin* __restrict__ qI, const float* __restrict__ w,
-    const Tin* __restrict__ KI, int64_t ldK, const int32_t* __restrict__ seq_of_q,
+    const Tin* __restrict__ KI, int64_t ldK, int nseq, const int32_t* __restrict__ seq_of_q,
     const int64_t* __restrict__ pos, const int64_t* __restrict__ n_entries, int H_I, int c_I,
     float* __restrict__ scores, int64_t ld_scores) {
   extern __shared__ float smem[];
   const int q = blockIdx.y;
   const int b = seq_of_q[q];
+  if (b < 0 || b >= nseq) return;
   const int64_t nv = n_visible(pos[q], g.m, g.vis_offset, min(n_entries[b], ldK));
   const int64_t s0 = (int64_t)blockIdx.x * 128;
   if (s0 >= nv) return;
@@ -105,7 +106,7 @@ __device__ int block_exclusive_scan(int v, int* sh, int* total) {
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(
     csa_geom g, const float* __restrict__ scores, int64_t ld_scores,
-    const int32_t* __restrict__ seq_of_q, const int64_t* __restrict__ pos,
+    int nseq, const int32_t* __restrict__ seq_of_q, const int64_t* __restrict__ pos,
     const int64_t* __restrict__ n_entries, int k, int32_t* __restrict__ idx_out,
     float* __restrict__ scores_dbg, int64_t ld_dbg) {
   __shared__ int hist[256];
@@ -114,7 +115,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(
   __shared__ int sh_remaining;
   const int q = blockIdx.x;
   const int b = seq_of_q[q];
-  const int64_t nv = n_visible(pos[q], g.m, g.vis_offset, min(n_entries[b], ld_scores));
+  const int64_t nv =
+      (b < 0 || b >= nseq) ? 0 : n_visible(pos[q], g.m, g.vis_offset, min(n_entries[b], ld_scores));
   const float* sc = scores + (int64_t)q * ld_scores;
   int32_t* out = idx_out + (int64_t)q * k;
   if (scores_dbg)
@@ -185,7 +187,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(
 
 template <typename Tin, int HMAX>
 static cudaError_t index_simt_t(const csa_geom& g, const void* qI, const float* w, const void* KI,
-                                int64_t ldK, const int32_t* seq_of_q, const int64_t* pos,
+                                int64_t ldK, int nseq, const int32_t* seq_of_q, const int64_t* pos,
                                 const int64_t* n_entries, int Q, int H_I, int c_I, float* scores,
                                 int64_t ld_scores, cudaStream_t s) {
   size_t smem = sizeof(float) * ((size_t)H_I * c_I + HMAX + 128 * (size_t)(c_I + 1));
@@ -195,22 +197,23 @@ static cudaError_t index_simt_t(const csa_geom& g, const void* qI, const float* 
   dim3 grid((unsigned)((ldK + 127) / 128), (unsigned)Q);
   count_launches();
   kern<<<grid, 128, smem, s>>>(g, reinterpret_cast<const Tin*>(qI), w,
-                               reinterpret_cast<const Tin*>(KI), ldK, seq_of_q, pos, n_entries,
+                               reinterpret_cast<const Tin*>(KI), ldK, nseq, seq_of_q, pos, n_entries,
                                H_I, c_I, scores, ld_scores);
   return cudaGetLastError();
 }
 
 cudaError_t launch_index_scores_simt(const csa_geom& g, int dt, const void* qI, const float* w,
-                                     const void* KI, int64_t ldK, const int32_t* seq_of_q,
+                                     const void* KI, int64_t ldK, int nseq,
+                                     const int32_t* seq_of_q,
                                      const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
                                      int c_I, float* scores, int64_t ld_scores, cudaStream_t s) {
   if (Q == 0 || ldK == 0) return cudaSuccess;
 #define CSA_IDX_CASE(HM)                                                                       \
   if (H_I <= HM)                                                                               \
     return dt == CSA_F32                                                                       \
-               ? index_simt_t<float, HM>(g, qI, w, KI, ldK, seq_of_q, pos, n_entries, Q, H_I,  \
+               ? index_simt_t<float, HM>(g, qI, w, KI, ldK, nseq, seq_of_q, pos, n_entries, Q, H_I,  \
                                          c_I, scores, ld_scores, s)                            \
-               : index_simt_t<__nv_bfloat16, HM>(g, qI, w, KI, ldK, seq_of_q, pos, n_entries,  \
+               : index_simt_t<__nv_bfloat16, HM>(g, qI, w, KI, ldK, nseq, seq_of_q, pos, n_entries,  \
                                                  Q, H_I, c_I, scores, ld_scores, s);
   CSA_IDX_CASE(8)
   CSA_IDX_CASE(32)
@@ -221,12 +224,12 @@ cudaError_t launch_index_scores_simt(const csa_geom& g, int dt, const void* qI, 
 }
 
 cudaError_t launch_topk_from_scores(const csa_geom& g, const float* scores, int64_t ld_scores,
-                                    const int32_t* seq_of_q, const int64_t* pos,
+                                    int nseq, const int32_t* seq_of_q, const int64_t* pos,
                                     const int64_t* n_entries, int Q, int k, int32_t* idx_out,
                                     float* scores_dbg, int64_t ld_dbg, cudaStream_t s) {
   if (Q == 0) return cudaSuccess;
   count_launches();
-  topk_kernel<<<Q, kTopkThreads, 0, s>>>(g, scores, ld_scores, seq_of_q, pos, n_entries, k,
+  topk_kernel<<<Q, kTopkThreads, 0, s>>>(g, scores, ld_scores, nseq, seq_of_q, pos, n_entries, k,
                                          idx_out, scores_dbg, ld_dbg);
   return cudaGetLastError();
 }

@@ -205,7 +205,8 @@ csa_status csa_compress_decode(const csa_geom* g, csa_dtype dtype, const void* h
  * with -1.
  *   qI        [Q, H_I, c_I] dtype (F32 or BF16)
  *   w         [Q, H_I] FP32
- *   KI        [nseq, ldK, c_I] dtype
+ *   KI        [nseq, ldK, c_I] dtype (queries whose seq_of_q is outside
+ *             [0, nseq) see no entries)
  *   seq_of_q  [Q] int32, pos [Q] int64, n_entries [nseq] int64 (device)
  *   idx_out   [Q, k] int32
  *   scores_dbg [Q, ldK] FP32 or NULL: when given, the kernel's FP32 scores
@@ -216,7 +217,7 @@ csa_status csa_compress_decode(const csa_geom* g, csa_dtype dtype, const void* h
  * --------------------------------------------------------------------- */
 size_t csa_index_topk_workspace_size(int Q, int64_t ldK, int k);
 csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, const float* w,
-                          const void* KI, int64_t ldK, const int32_t* seq_of_q,
+                          const void* KI, int64_t ldK, int nseq, const int32_t* seq_of_q,
                           const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
                           int c_I, int k, int32_t* idx_out, float* scores_dbg,
                           void* workspace, size_t ws_bytes, csa_stream_t stream);
@@ -235,7 +236,8 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
  *   O[q,h,:] = o with its last rope_dims dims rotated by -p.
  *   q     [Q, H_q, c] q_dtype (F32 or BF16); O [Q, H_q, c] q_dtype
  *   q_gain [c] FP32 or NULL (ones); sink [H_q] FP32
- *   E     [nseq, ldE, c] kv_dtype (F32, BF16, or mixed rows)
+ *   E     [nseq, ldE, c] kv_dtype (F32, BF16, or mixed rows); queries whose
+ *         seq_of_q is outside [0, nseq) produce zeros
  *   idx   [Q, k] int32, entries < n_entries[b] or -1 (slots holding -1 or
  *         an index >= ldE are skipped)
  *   win   [nseq, ldW, c] kv_dtype (F32 or BF16), rows already prepared
@@ -246,7 +248,7 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win);
 csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,
                       const float* q_gain, const float* sink, const void* E, int64_t ldE,
-                      const int64_t* n_entries, const int32_t* idx, int k, const void* win,
+                      int nseq, const int64_t* n_entries, const int32_t* idx, int k, const void* win,
                       int64_t ldW, const int32_t* seq_of_q, const int64_t* pos, int Q, int H_q,
                       void* O, void* workspace, size_t ws_bytes, csa_stream_t stream);
 
@@ -260,7 +262,7 @@ csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, 
 size_t hca_attend_workspace_size(int Q, int H_q, int c, int64_t ldE, int n_win);
 csa_status hca_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,
                       const float* q_gain, const float* sink, const void* E, int64_t ldE,
-                      const int64_t* n_entries, const void* win, int64_t ldW,
+                      int nseq, const int64_t* n_entries, const void* win, int64_t ldW,
                       const int32_t* seq_of_q, const int64_t* pos, int Q, int H_q, void* O,
                       void* workspace, size_t ws_bytes, csa_stream_t stream);
 

@@ -79,8 +79,8 @@ def test_null_and_misaligned_pointers_rejected(lib):
 
 def test_index_topk_argument_checks(lib):
     g = csa.geom()
-    args = lambda k, HI, cI, ws, wsb: (ctypes.byref(g), 1, OK, OK, OK, 100, OK, OK, OK, 4, HI, cI,
-                                       k, OK, None, ws, wsb, None)
+    args = lambda k, HI, cI, ws, wsb: (ctypes.byref(g), 1, OK, OK, OK, 100, 1, OK, OK, OK, 4, HI,
+                                       cI, k, OK, None, ws, wsb, None)
     assert lib.csa_index_topk(*args(0, 64, 128, OK, 1 << 20)) == 1      # k = 0
     assert lib.csa_index_topk(*args(4096, 64, 128, OK, 1 << 20)) == 1   # k > max
     assert lib.csa_index_topk(*args(16, 64, 100, OK, 1 << 20)) == 1     # c_I % 16
@@ -105,9 +105,9 @@ def test_compress_argument_checks(lib):
 def test_attend_argument_checks(lib):
     g = csa.geom(win_ring=1)
     # ring window with fewer rows than n_win
-    assert lib.csa_attend(ctypes.byref(g), 1, 1, OK, None, OK, OK, 10, OK, OK, 8, OK, 64, OK, OK,
-                          2, 64, OK, None, 0, None) == 1
+    assert lib.csa_attend(ctypes.byref(g), 1, 1, OK, None, OK, OK, 10, 1, OK, OK, 8, OK, 64, OK,
+                          OK, 2, 64, OK, None, 0, None) == 1
     # bad q dtype
     g0 = csa.geom()
-    assert lib.csa_attend(ctypes.byref(g0), 2, 1, OK, None, OK, OK, 10, OK, OK, 8, OK, 500, OK,
+    assert lib.csa_attend(ctypes.byref(g0), 2, 1, OK, None, OK, OK, 10, 1, OK, OK, 8, OK, 500, OK,
                           OK, 2, 64, OK, None, 0, None) == 1
