@@ -203,8 +203,8 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
 }
 
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win) {
-  (void)Q; (void)H_q; (void)c; (void)k; (void)n_win;
-  return 0;
+  if (Q <= 0 || k < 0 || n_win < 0 || c != 512 || H_q != 64) return 0;
+  return csa::attend_tc_workspace(Q, (int64_t)k + n_win);
 }
 
 static csa_status attend_common(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype,
@@ -212,7 +212,8 @@ static csa_status attend_common(const csa_geom* g, csa_dtype q_dtype, csa_dtype 
                                 const void* E, int64_t ldE, int nseq, const int64_t* n_entries,
                                 const int32_t* idx, int k, int dense, const void* win,
                                 int64_t ldW, const int32_t* seq_of_q, const int64_t* pos, int Q,
-                                int H_q, void* O, csa_stream_t stream) {
+                                int H_q, void* O, void* workspace, size_t ws_bytes,
+                                csa_stream_t stream) {
   if (!geom_ok(g) || !io_dtype_ok(q_dtype)) return CSA_ERR_INVALID_ARG;
   if (!(io_dtype_ok(kv_dtype) || (kv_dtype == CSA_FP8_MIXED && mixed_ok(g)))) return CSA_ERR_INVALID_ARG;
   if (Q < 0 || H_q < 1 || ldE < 0 || ldW < 0 || nseq < 0) return CSA_ERR_INVALID_ARG;
@@ -225,6 +226,16 @@ static csa_status attend_common(const csa_geom* g, csa_dtype q_dtype, csa_dtype 
   const void* ptrs[] = {q, q_gain, sink, E, n_entries, idx, win, seq_of_q, pos, O};
   for (const void* p : ptrs)
     if (!aligned16(p)) return CSA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return CSA_ERR_INVALID_ARG;
+  if (csa::attend_tc_supported(q_dtype, kv_dtype, g->c, H_q, dense ? 0 : k, g->rope_dims)) {
+    const int64_t max_slots = (dense ? ldE : (int64_t)k) + g->n_win;
+    const size_t need = csa::attend_tc_workspace(Q, max_slots);
+    if (need > 0 && (!workspace || ws_bytes < need)) return CSA_ERR_INVALID_ARG;
+    return cuda_status(csa::launch_attend_tc(*g, kv_dtype, q, q_gain, sink, E, ldE, nseq, n_entries,
+                                             idx, dense ? 0 : k, dense, win, ldW, seq_of_q, pos, Q,
+                                             O, workspace, ws_bytes,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+  }
   if (!csa::attend_simt_supported(g->c, H_q)) return CSA_ERR_UNSUPPORTED;
   return cuda_status(launch_attend_simt(*g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, nseq,
                                         n_entries, idx, k, dense, win, ldW, seq_of_q, pos, Q, H_q, O,
@@ -237,16 +248,13 @@ csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, 
                       const void* win, int64_t ldW, const int32_t* seq_of_q, const int64_t* pos,
                       int Q, int H_q, void* O, void* workspace, size_t ws_bytes,
                       csa_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
   return attend_common(g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, nseq, n_entries, idx, k, 0,
-                       win,
-                       ldW, seq_of_q, pos, Q, H_q, O, stream);
+                       win, ldW, seq_of_q, pos, Q, H_q, O, workspace, ws_bytes, stream);
 }
 
 size_t hca_attend_workspace_size(int Q, int H_q, int c, int64_t ldE, int n_win) {
-  (void)Q; (void)H_q; (void)c; (void)ldE; (void)n_win;
-  return 0;
+  if (Q <= 0 || ldE < 0 || n_win < 0 || c != 512 || H_q != 64) return 0;
+  return csa::attend_tc_workspace(Q, ldE + n_win);
 }
 
 csa_status hca_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,
@@ -254,11 +262,8 @@ csa_status hca_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, 
                       int nseq, const int64_t* n_entries, const void* win, int64_t ldW,
                       const int32_t* seq_of_q, const int64_t* pos, int Q, int H_q, void* O,
                       void* workspace, size_t ws_bytes, csa_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
   return attend_common(g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, nseq, n_entries, nullptr, 0,
-                       1,
-                       win, ldW, seq_of_q, pos, Q, H_q, O, stream);
+                       1, win, ldW, seq_of_q, pos, Q, H_q, O, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -51,6 +51,14 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
                                    const int32_t* seq_of_q, const int64_t* pos,
                                    const int64_t* n_entries, int Q, int H_I, int c_I,
                                    float* scores, int64_t ld_scores, cudaStream_t s);
+bool attend_tc_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_dims);
+size_t attend_tc_workspace(int Q, int64_t max_slots);
+cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,
+                             const float* sink, const void* E, int64_t ldE, int nseq,
+                             const int64_t* n_entries, const int32_t* idx, int k, int dense,
+                             const void* win, int64_t ldW, const int32_t* seq_of_q,
+                             const int64_t* pos, int Q, void* O, void* workspace,
+                             size_t ws_bytes, cudaStream_t s);
 // dense != 0: HCA (all visible entries); else CSA with idx [Q, k].
 cudaError_t launch_attend_simt(const csa_geom& g, int q_dt, int kv_dt, const void* q,
                                const float* q_gain, const float* sink, const void* E,

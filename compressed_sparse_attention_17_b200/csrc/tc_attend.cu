@@ -1,0 +1,564 @@
+// tc_attend.cu - shared-KV multi-query core attention on the 5th-generation
+// tensor cores: compressed entries (selected by the indexer, or every
+// visible one for HCA) plus the sliding window, one softmax whose
+// denominator carries the sink, RMSNorm + RoPE on the queries and inverse
+// RoPE on the outputs ("Evidence Ledger", CSA Eqs 18-19, Shared attention
+// details Sec 2.3.3 and Eq 27; "DeepSeek-V4" study 03).
+//
+// Orientation. One CTA serves one query token (all 64 heads). Keys are
+// gathered 128 at a time into a 128-byte-swizzled K-major tile
+// sK[key][dim]; the heads are the MMA's N dimension:
+//   S^T[key, head]  = sK (K-major A, K = dims) x Qhat (K-major B)
+//   O^T[dim, head] += sK^T (MN-major A, K = keys) x P^T (MN-major B)
+// so the one shared-memory tile is both K and V, as the shared-KV MQA
+// prescribes. S^T takes 64 TMEM columns, O^T 4 x 64 (512 dims).
+//
+// Softmax. Each epilogue thread owns one key (TMEM lane) and its 64 head
+// logits. The per-head reference value m_h starts at the sink logit and is
+// raised only when a tile's maximum exceeds it by more than 2^8 (then O^T
+// and the running sums are rescaled): every weight exp(l - m_h) stays below
+// 2^8, so the FP32 sums and the BF16 weights neither overflow nor lose
+// range, and the result is the exact softmax up to rounding.
+//
+// Small batches split each query's key list across CTAs (fixed split
+// boundaries) and merge the partial (m, l, O) in a fixed order, so a
+// query's result does not depend on the batch it is in.
+//
+// Warps (288 threads): 0-3 gather key rows (cp.async) and prepare Qhat with
+// 4-7; 4-7 run the softmax and the output epilogue (TMEM lane quadrant =
+// warp % 4); 8 owns TMEM and issues the MMAs.
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kThreads = 288;
+constexpr int kHeads = 64;
+constexpr int kDim = 512;
+constexpr int kTile = 128;          // keys per tile
+constexpr int kChunks = kDim / 64;  // 64-dim chunks of a key row
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;       // S^T: 64 columns
+constexpr uint32_t kColO = 256;     // O^T: 4 blocks x 64 columns
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;
+
+// shared memory map (offsets from the 1024-aligned base)
+constexpr int kOffK = 0;                           // 8 x 16 KB
+constexpr int kOffQ = kOffK + kChunks * 16384;     // 8 x 8 KB
+constexpr int kOffP = kOffQ + kChunks * 8192;      // 16 KB
+constexpr int kOffRed = kOffP + 16384;             // 4 x 64 floats
+constexpr int kOffRef = kOffRed + 4 * kHeads * 4;  // 64 floats (log2 units)
+constexpr int kOffAlpha = kOffRef + kHeads * 4;    // 64 floats
+constexpr int kOffMisc = kOffAlpha + kHeads * 4;   // barriers, tmem slot, flags
+constexpr int kOffList = kOffMisc + 64;            // compacted entry list
+constexpr int kSmemFixed = kOffList + 1024;        // + alignment slack
+
+struct Params {
+  int Q, r, m, vis_offset, n_win, win_ring, kv_dt, k, dense, nseq;
+  double base;
+  float eps;
+  const __nv_bfloat16* q;
+  const float* q_gain;
+  const float* sink;
+  const void* E;
+  int64_t ldE;
+  const int64_t* n_entries;
+  const int32_t* idx;
+  const __nv_bfloat16* win;
+  int64_t ldW;
+  const int32_t* seq_of_q;
+  const int64_t* pos;
+  __nv_bfloat16* O;
+  int tiles_per_split;  // 0: one CTA per query does every tile
+  int max_splits;
+  float* part_O;        // [Q][max_splits][64][512]
+  float* part_ml;       // [Q][max_splits][64][2]: reference (log2 units), sum
+  int* err;
+};
+
+__device__ __forceinline__ int order_int(float f) {
+  int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float from_order_int(int i) {
+  return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const uint32_t sK = tc::smem_u32(sm + kOffK);
+  const uint32_t sQ = tc::smem_u32(sm + kOffQ);
+  const uint32_t sP = tc::smem_u32(sm + kOffP);
+  float* red = reinterpret_cast<float*>(sm + kOffRed);
+  float* ref2 = reinterpret_cast<float*>(sm + kOffRef);
+  float* alpha = reinterpret_cast<float*>(sm + kOffAlpha);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffMisc);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kOffMisc + 16);
+  int* flags = reinterpret_cast<int*>(sm + kOffMisc + 32);  // [0] abort, [1] rescale, [2] nvalid
+  int32_t* list = reinterpret_cast<int32_t*>(sm + kOffList);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qi = blockIdx.y;
+  const int split = blockIdx.x;
+  const int b = P.seq_of_q[qi];
+  const int64_t p = P.pos[qi];
+  const bool valid_seq = b >= 0 && b < P.nseq;
+  const uint32_t s_bar = tc::smem_u32(&bars[0]);
+  const uint32_t o_bar = tc::smem_u32(&bars[1]);
+
+  // ---- setup: barriers, TMEM, compacted entry list ----
+  if (threadIdx.x == 0) {
+    tc::mbar_init(s_bar, 1);
+    tc::mbar_init(o_bar, 1);
+    flags[0] = 0;
+    flags[1] = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 8) tc::tmem_alloc(tc::smem_u32(tslot), kTmemCols);
+  const int64_t ldE = P.ldE;
+  int64_t nsel = 0;
+  if (valid_seq) {
+    if (P.dense) {
+      nsel = n_visible(p, P.m, P.vis_offset, min(P.n_entries[b], ldE));
+    } else {
+      // keep the slots that hold an entry inside the cache, in order
+      if (warp < 8) {
+        const int32_t* row = P.idx + (int64_t)qi * P.k;
+        __shared__ int wcount[8];
+        int base_total = 0;
+        for (int j0 = 0; j0 < P.k; j0 += 256) {
+          const int j = j0 + threadIdx.x;
+          const int32_t e = j < P.k ? row[j] : -1;
+          const bool ok = e >= 0 && e < ldE;
+          const unsigned msk = __ballot_sync(0xffffffffu, ok);
+          if (lane == 0) wcount[warp] = __popc(msk);
+          tc::named_bar(2, 256);
+          int before = 0, tot = 0;
+          for (int w = 0; w < 8; ++w) {
+            before += w < warp ? wcount[w] : 0;
+            tot += wcount[w];
+          }
+          if (ok) list[base_total + before + __popc(msk & ((1u << lane) - 1u))] = e;
+          base_total += tot;
+          tc::named_bar(2, 256);
+        }
+        if (threadIdx.x == 0) flags[2] = base_total;
+      }
+    }
+  }
+  // ---- q-hat = RoPE_p(RMSNorm(q_h) * gain) in BF16, K-major swizzled ----
+  if (valid_seq && warp < 8) {
+    for (int h = warp; h < kHeads; h += 8) {
+      const __nv_bfloat16* qr = P.q + ((int64_t)qi * kHeads + h) * kDim;
+      float v[16];
+      const uint4* src = reinterpret_cast<const uint4*>(qr + 16 * lane);
+      uint4 u0 = src[0], u1 = src[1];
+      const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&u0);
+      const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&u1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 a = __bfloat1622float2(h0[i]), c2 = __bfloat1622float2(h1[i]);
+        v[2 * i] = a.x;
+        v[2 * i + 1] = a.y;
+        v[8 + 2 * i] = c2.x;
+        v[8 + 2 * i + 1] = c2.y;
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ss += v[i] * v[i];
+      ss = warp_sum(ss);
+      const float inv = 1.f / sqrtf(ss / (float)kDim + P.eps);
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        const int d = 16 * lane + i;
+        float a = v[i] * inv * (P.q_gain ? P.q_gain[d] : 1.f);
+        float bb = v[i + 1] * inv * (P.q_gain ? P.q_gain[d + 1] : 1.f);
+        if (d >= kDim - P.r) {
+          float cs, sn;
+          rope_cs(p, (d - (kDim - P.r)) >> 1, P.r, P.base, &cs, &sn);
+          const float a2 = a * cs - bb * sn;
+          bb = a * sn + bb * cs;
+          a = a2;
+        }
+        v[i] = a;
+        v[i + 1] = bb;
+      }
+      // dims 16*lane .. +15 = granules 2*lane, 2*lane+1 of chunk lane/4
+      const int chunk = lane >> 2;
+#pragma unroll
+      for (int gq = 0; gq < 2; ++gq) {
+        const uint32_t g = (uint32_t)((2 * lane + gq) & 7);
+        __nv_bfloat162 pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pk[i] = __floats2bfloat162_rn(v[8 * gq + 2 * i], v[8 * gq + 2 * i + 1]);
+        const uint32_t dst = sQ + chunk * 8192 + tc::sw128_offset((uint32_t)h, g);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                     "r"(*reinterpret_cast<uint32_t*>(&pk[0])), "r"(*reinterpret_cast<uint32_t*>(&pk[1])),
+                     "r"(*reinterpret_cast<uint32_t*>(&pk[2])), "r"(*reinterpret_cast<uint32_t*>(&pk[3]))
+                     : "memory");
+      }
+    }
+  }
+  if (threadIdx.x < kHeads) ref2[threadIdx.x] = P.sink[threadIdx.x] * kLog2e;
+  tc::fence_proxy_async();
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  if (valid_seq && !P.dense) nsel = flags[2];
+
+  // ---- key slots of this CTA ----
+  const int64_t w0 = p - P.n_win + 1 > 0 ? p - P.n_win + 1 : 0;
+  const int64_t nwin = (valid_seq && P.n_win > 0) ? p - w0 + 1 : 0;
+  const int64_t nslots = valid_seq ? nsel + nwin : 0;
+  const int64_t ntiles = (nslots + kTile - 1) / kTile;
+  int64_t t_begin = 0, t_end = ntiles;
+  if (P.tiles_per_split > 0) {
+    t_begin = (int64_t)split * P.tiles_per_split;
+    t_end = min(ntiles, t_begin + P.tiles_per_split);
+  }
+  const float scale2 = kLog2e / sqrtf((float)kDim);
+  float lsum[kHeads];
+#pragma unroll
+  for (int h = 0; h < kHeads; ++h) lsum[h] = 0.f;
+  const int row_bytes_e = (int)row_bytes(P.kv_dt, kDim);
+
+  uint32_t phase = 0;
+  for (int64_t t = t_begin; t < t_end; ++t) {
+    // ---- gather 128 key rows into sK (warps 0-3, one row per warp-step) ----
+    if (warp < 4) {
+      for (int rr = warp; rr < kTile; rr += 4) {
+        const int64_t slot = t * kTile + rr;
+        const uint8_t* row = nullptr;
+        bool mixed = false;
+        if (slot < nslots) {
+          if (slot < nsel) {
+            const int64_t e = P.dense ? slot : (int64_t)list[slot];
+            row = reinterpret_cast<const uint8_t*>(P.E) + ((int64_t)b * ldE + e) * row_bytes_e;
+            mixed = P.kv_dt == CSA_FP8_MIXED;
+          } else {
+            const int64_t j = w0 + (slot - nsel);
+            const int64_t wr = P.win_ring ? (j % P.n_win) : j;
+            if (wr < P.ldW)
+              row = reinterpret_cast<const uint8_t*>(P.win + ((int64_t)b * P.ldW + wr) * kDim);
+          }
+        }
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          const int g = lane + 32 * gg;  // 16-byte granule of the row: dims 8g .. 8g+7
+          const uint32_t dst = sK + (g >> 3) * 16384 + tc::sw128_offset((uint32_t)rr, (uint32_t)(g & 7));
+          if (row == nullptr) {
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+          } else if (!mixed) {
+            tc::cp_async16(dst, row + 16 * g);
+          } else {
+            uint32_t o[4];
+            if (8 * g < kMixedFp8Dims) {
+              const float sc = *reinterpret_cast<const float*>(row + kMixedScaleOffset);
+              const uint2 codes = *reinterpret_cast<const uint2*>(row + 8 * g);
+              const uint8_t* cb = reinterpret_cast<const uint8_t*>(&codes);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                __nv_bfloat162 pr = __floats2bfloat162_rn(e4m3_to_f32(cb[2 * i]) * sc,
+                                                          e4m3_to_f32(cb[2 * i + 1]) * sc);
+                o[i] = *reinterpret_cast<uint32_t*>(&pr);
+              }
+            } else {
+              const uint4 v = *reinterpret_cast<const uint4*>(row + kMixedFp8Dims + 2 * (8 * g - kMixedFp8Dims));
+              o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+            }
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]),
+                         "r"(o[2]), "r"(o[3])
+                         : "memory");
+          }
+        }
+      }
+      tc::cp_async_wait_all();
+      tc::fence_proxy_async();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+
+    // ---- S^T = K Qhat^T ----
+    if (warp == 8 && lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(128, kHeads);
+      for (int kk = 0; kk < kDim / 16; ++kk) {
+        const uint32_t ch = kk >> 2, off = (uint32_t)(kk & 3) * 32;
+        tc::mma_bf16(tmem + kColS, tc::sdesc_kmajor_sw128(sK + ch * 16384 + off),
+                     tc::sdesc_kmajor_sw128(sQ + ch * 8192 + off), idesc, kk > 0);
+      }
+      tc::mma_commit(s_bar);
+    }
+    // ---- softmax on the key lanes ----
+    if (warp >= 4 && warp < 8) {
+      const int quad = warp & 3;
+      const int key = quad * 32 + lane;
+      const int64_t slot = t * kTile + key;
+      const bool kvalid = slot < nslots;
+      float s[kHeads];
+      const bool ok = tc::mbar_wait(s_bar, phase, P.err);
+      if (!ok) flags[0] = 1;
+      tc::tc_fence_after();
+      tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + kColS, s);
+      tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + kColS + 32, s + 32);
+#pragma unroll
+      for (int h = 0; h < kHeads; ++h) s[h] = kvalid ? s[h] * scale2 : -INFINITY;
+      // per-head maximum over the 128 keys
+#pragma unroll
+      for (int h = 0; h < kHeads; ++h) {
+        const int mx = __reduce_max_sync(0xffffffffu, order_int(s[h]));
+        if (lane == 0) red[quad * kHeads + h] = from_order_int(mx);
+      }
+      tc::named_bar(1, 128);
+      if (warp == 4 || warp == 5) {
+        const int h = (warp - 4) * 32 + lane;
+        const float tmax = fmaxf(fmaxf(red[h], red[kHeads + h]), fmaxf(red[2 * kHeads + h], red[3 * kHeads + h]));
+        float a = 1.f;
+        if (tmax > ref2[h] + kRescaleLog2) {
+          a = exp2f(ref2[h] - tmax);
+          ref2[h] = tmax;
+          flags[1] = 1;
+        }
+        alpha[h] = a;
+      }
+      tc::named_bar(1, 128);
+      // weights in BF16, one 128-byte row per key (heads contiguous)
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int h = 8 * g + 2 * i;
+          const float p0 = exp2f(s[h] - ref2[h]), p1 = exp2f(s[h + 1] - ref2[h + 1]);
+          lsum[h] = lsum[h] * alpha[h] + p0;
+          lsum[h + 1] = lsum[h + 1] * alpha[h + 1] + p1;
+          __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+          pk[i] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sP + tc::sw128_offset((uint32_t)key, (uint32_t)g)),
+                     "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                     : "memory");
+      }
+      // rescale the accumulated O^T (this thread's dim lane in each block)
+      if (flags[1] && t > t_begin) {
+        const float* al = alpha;
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < kHeads; c0 += 32) {
+            float o[32];
+            const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + kColO + blk * kHeads + c0;
+            tc::tmem_ld32(ta, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= al[c0 + i];
+            tc::tmem_st32(ta, o);
+          }
+        }
+      }
+      tc::fence_proxy_async();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (threadIdx.x == 0) flags[1] = 0;
+    // ---- O^T += K^T P^T ----
+    if (warp == 8 && lane == 0) {
+      if (!flags[0]) {
+        const uint32_t idesc = tc::idesc_bf16_f32_major(128, kHeads, 1, 1);
+        for (int blk = 0; blk < 4; ++blk) {
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t ad = tc::sdesc_mnmajor_sw128(sK + (2 * blk) * 16384 + kk * 2048, 16384, 1024);
+            const uint64_t bd = tc::sdesc_mnmajor_sw128(sP + kk * 2048, 8192, 1024);
+            tc::mma_bf16(tmem + kColO + blk * kHeads, ad, bd, idesc, (t > t_begin || kk > 0) ? 1u : 0u);
+          }
+        }
+      }
+      tc::mma_commit(o_bar);
+    }
+    if (!tc::mbar_wait(o_bar, phase, P.err)) flags[0] = 1;
+    tc::tc_fence_after();
+    phase ^= 1u;
+    __syncthreads();
+    if (flags[0]) break;
+  }
+
+  // ---- epilogue: sums over keys, normalisation, inverse RoPE, store ----
+  const bool have = t_end > t_begin && !flags[0];
+  if (warp >= 4 && warp < 8) {
+    const int quad = warp & 3;
+    // per-head sum of the weights over the 128 key lanes
+    for (int h = 0; h < kHeads; ++h) {
+      float v = warp_sum(lsum[h]);
+      if (lane == 0) red[quad * kHeads + h] = v;
+    }
+    tc::named_bar(1, 128);
+    const int dim_in_blk = quad * 32 + lane;
+    const bool split_mode = P.tiles_per_split > 0;
+    for (int blk = 0; blk < 4; ++blk) {
+      const int d = blk * 128 + dim_in_blk;
+      float cs = 1.f, sn = 0.f;
+      const bool rot = d >= kDim - P.r;
+      if (rot && !split_mode) rope_cs(p, (d - (kDim - P.r)) >> 1, P.r, P.base, &cs, &sn);
+      for (int c0 = 0; c0 < kHeads; c0 += 32) {
+        float o[32];
+        if (have) {
+          tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + kColO + blk * kHeads + c0, o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int h = c0 + i;
+          const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
+          if (split_mode) {
+            P.part_O[(((int64_t)qi * P.max_splits + split) * kHeads + h) * kDim + d] = have ? o[i] : 0.f;
+          } else {
+            const float den = l + exp2f(P.sink[h] * kLog2e - ref2[h]);
+            float val = valid_seq ? o[i] / den : 0.f;
+            if (rot) {
+              // pair (d, d^1) sits in the neighbouring lane; rotate by -p
+              const float other = __shfl_xor_sync(0xffffffffu, val, 1);
+              val = (d & 1) ? (-other * sn + val * cs) : (val * cs + other * sn);
+            }
+            P.O[((int64_t)qi * kHeads + h) * kDim + d] = __float2bfloat16_rn(val);
+          }
+        }
+      }
+    }
+    if (split_mode && warp == 4) {
+      for (int h = lane; h < kHeads; h += 32) {
+        const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
+        float* ml = P.part_ml + (((int64_t)qi * P.max_splits + split) * kHeads + h) * 2;
+        ml[0] = ref2[h];
+        ml[1] = have ? l : 0.f;
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 8) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// Merge of split partials: O = sum_s O_s 2^(m_s - m) / (2^(z'log2e - m) +
+// sum_s l_s 2^(m_s - m)), m the largest reference, fixed split order; then
+// inverse RoPE and the BF16 store. One block per (query, head).
+__global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
+  const int qi = blockIdx.x / kHeads, h = blockIdx.x % kHeads;
+  const int b = P.seq_of_q[qi];
+  const int64_t p = P.pos[qi];
+  const float* ml = P.part_ml + ((int64_t)qi * P.max_splits * kHeads + h) * 2;
+  const float z2 = P.sink[h] * kLog2e;
+  float m = z2;
+  for (int sp = 0; sp < P.max_splits; ++sp) m = fmaxf(m, ml[(int64_t)sp * kHeads * 2]);
+  float den = exp2f(z2 - m);
+  for (int sp = 0; sp < P.max_splits; ++sp)
+    den += ml[(int64_t)sp * kHeads * 2 + 1] * exp2f(ml[(int64_t)sp * kHeads * 2] - m);
+  const bool valid_seq = b >= 0 && b < P.nseq;
+  for (int d0 = 2 * threadIdx.x; d0 < kDim; d0 += 256) {
+    float a = 0.f, c = 0.f;
+    for (int sp = 0; sp < P.max_splits; ++sp) {
+      const float wgt = exp2f(ml[(int64_t)sp * kHeads * 2] - m);
+      const float* po = P.part_O + (((int64_t)qi * P.max_splits + sp) * kHeads + h) * kDim + d0;
+      a = fmaf(po[0], wgt, a);
+      c = fmaf(po[1], wgt, c);
+    }
+    a = valid_seq ? a / den : 0.f;
+    c = valid_seq ? c / den : 0.f;
+    if (d0 >= kDim - P.r) {
+      float cs, sn;
+      rope_cs(p, (d0 - (kDim - P.r)) >> 1, P.r, P.base, &cs, &sn);
+      const float a2 = a * cs + c * sn;
+      c = -a * sn + c * cs;
+      a = a2;
+    }
+    __nv_bfloat162 pr = __floats2bfloat162_rn(a, c);
+    *reinterpret_cast<__nv_bfloat162*>(P.O + ((int64_t)qi * kHeads + h) * kDim + d0) = pr;
+  }
+}
+
+int choose_tiles_per_split(int Q, int64_t max_slots) {
+  const int64_t tiles = (max_slots + kTile - 1) / kTile;
+  // few queries: one tile per CTA so that every SM has work
+  return ((int64_t)Q * tiles <= 4 * 148) ? 1 : 0;
+}
+
+}  // namespace
+
+bool attend_tc_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_dims) {
+  return q_dt == CSA_BF16 && (kv_dt == CSA_BF16 || kv_dt == CSA_FP8_MIXED) && c == kDim &&
+         H_q == kHeads && k <= CSA_MAX_TOPK && rope_dims % 32 == 0;
+}
+
+size_t attend_tc_workspace(int Q, int64_t max_slots) {
+  const int tps = choose_tiles_per_split(Q, max_slots);
+  if (tps == 0) return 0;
+  const int64_t splits = (max_slots + kTile - 1) / kTile;
+  return (size_t)Q * splits * kHeads * ((size_t)kDim + 2) * sizeof(float);
+}
+
+cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,
+                             const float* sink, const void* E, int64_t ldE, int nseq,
+                             const int64_t* n_entries, const int32_t* idx, int k, int dense,
+                             const void* win, int64_t ldW, const int32_t* seq_of_q,
+                             const int64_t* pos, int Q, void* O, void* workspace,
+                             size_t ws_bytes, cudaStream_t s) {
+  if (Q == 0) return cudaSuccess;
+  const int64_t max_slots = (dense ? ldE : (int64_t)k) + g.n_win;
+  Params P{};
+  P.Q = Q;
+  P.r = g.rope_dims;
+  P.m = g.m;
+  P.vis_offset = g.vis_offset;
+  P.n_win = g.n_win;
+  P.win_ring = g.win_ring;
+  P.kv_dt = kv_dt;
+  P.k = k;
+  P.dense = dense;
+  P.nseq = nseq;
+  P.base = g.rope_base;
+  P.eps = g.eps;
+  P.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  P.q_gain = q_gain;
+  P.sink = sink;
+  P.E = E;
+  P.ldE = ldE;
+  P.n_entries = n_entries;
+  P.idx = idx;
+  P.win = reinterpret_cast<const __nv_bfloat16*>(win);
+  P.ldW = ldW;
+  P.seq_of_q = seq_of_q;
+  P.pos = pos;
+  P.O = reinterpret_cast<__nv_bfloat16*>(O);
+  P.err = device_error_ptr();
+  P.tiles_per_split = choose_tiles_per_split(Q, max_slots);
+  int splits = 1;
+  if (P.tiles_per_split > 0) {
+    splits = (int)((max_slots + kTile - 1) / kTile);
+    if (ws_bytes < attend_tc_workspace(Q, max_slots) || workspace == nullptr)
+      return cudaErrorInvalidValue;
+    P.part_O = reinterpret_cast<float*>(workspace);
+    P.part_ml = P.part_O + (size_t)Q * splits * kHeads * kDim;
+  }
+  P.max_splits = splits;
+  const size_t smem = (size_t)kSmemFixed + (dense ? 0 : (size_t)k * 4) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  if (Q > 65535) return cudaErrorInvalidValue;
+  count_launches();
+  attend_tc_kernel<<<dim3((unsigned)splits, (unsigned)Q), kThreads, smem, s>>>(P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || P.tiles_per_split == 0) return e;
+  count_launches();
+  attend_merge_kernel<<<Q * kHeads, 128, 0, s>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -243,7 +243,9 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
  *   win   [nseq, ldW, c] kv_dtype (F32 or BF16), rows already prepared
  *         (csa_rmsnorm_rope); row of position j = j (win_ring = 0, ldW > p)
  *         or j mod n_win (win_ring = 1, ldW >= n_win).
- * workspace: csa_attend_workspace_size() bytes.
+ * workspace: csa_attend_workspace_size() bytes (non-zero when few queries
+ * are spread over more CTAs than one per query: the per-split partial
+ * results live there).
  * --------------------------------------------------------------------- */
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win);
 csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,

@@ -297,6 +297,40 @@ def test_hca_attend(orc, dt, m):
     assert max_abs(host(O), want) <= TOL[dt]
 
 
+@pytest.mark.parametrize("Q,k,hole", [(80, 1024, 0.05), (20, 300, 0.3)])
+def test_csa_attend_tensor_core_paths(orc, Q, k, hole):
+    """64 heads x 512 in BF16 run on the tensor-core kernel: many queries use
+    one CTA per query, few queries split the keys over CTAs and merge."""
+    Hq, c, r, N = 64, 512, 64, 1500
+    q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(orc, Q, Hq, c, r, 2, N, k, "bf16",
+                                                            ring=False, seed=21, hole=hole)
+    g = csa.geom(c=c, rope_dims=r)
+    O = csa.attend(dev(q, "bf16"), dev(sink, "f32"), dev(E, "bf16"), dev_i(idx, torch.int32),
+                   dev(win, "bf16"), dev_i(seq, torch.int32), dev_i(pos), dev_i(ne), g,
+                   q_gain=dev(gain, "f32"))
+    want = orc.attend(q, sink, E, win, seq, pos, ne, rope_dims=r, idx=idx, q_gain=gain)
+    assert max_abs(host(O), want) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("Q", [24, 300])
+def test_hca_attend_tensor_core_paths(orc, Q):
+    Hq, c, r, N, m = 64, 512, 64, 40, 128
+    rg = np.random.default_rng(31)
+    q = _spec("qh", (Q, Hq, c), 1.0, "bf16", 31).values()
+    E = _spec("Eh", (2, N, c), 1.0, "bf16", 31).values()
+    sink = _spec("sh", (Hq,), 1.0, "f32", 31).values()
+    seq = rg.integers(0, 2, Q).astype(np.int32)
+    pos = rg.integers(0, m * N + 300, Q).astype(np.int64)
+    pos[:3] = [0, 126, 127]
+    ne = np.array([N, N - 3])
+    win = _spec("wh", (2, int(pos.max()) + 1, c), 1.0, "bf16", 31).values()
+    g = csa.geom(m=m, overlap=0, c=c, rope_dims=r)
+    O = csa.hca_attend(dev(q, "bf16"), dev(sink, "f32"), dev(E, "bf16"), dev(win, "bf16"),
+                       dev_i(seq, torch.int32), dev_i(pos), dev_i(ne), g)
+    want = orc.attend(q, sink, E, win, seq, pos, ne, rope_dims=r, m=m)
+    assert max_abs(host(O), want) <= TOL["bf16"]
+
+
 def test_csa_attend_mixed_entries(orc):
     Q, Hq, c, r, N, k = 9, 64, 512, 64, 200, 64
     q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(orc, Q, Hq, c, r, 2, N, k, "bf16",
