@@ -80,7 +80,7 @@ class Clocks:
     def __enter__(self):
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                       "--format=csv,noheader,nounits", "-lms", "20"],
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
@@ -242,6 +242,32 @@ class Prefill:
                    self.g, out=self.O)
 
 
+class HcaPrefill:
+    """HCA prefill: non-overlapping m'=128 compressor, window preparation,
+    dense attention over every visible entry plus the window."""
+
+    def __init__(self, w: synth.Workload, device):
+        self.w, self.dev = w, device
+        t0 = time.time()
+        s = w.specs()
+        self.g = csa.geom(m=w.m, overlap=0, c=w.c, rope_dims=w.rope_dims)
+        self.t = {n: to_dev(s[n], device) for n in s}
+        T = w.T
+        self.pos = torch.arange(T, dtype=torch.int64, device=device)
+        self.seq = torch.zeros(T, dtype=torch.int32, device=device)
+        self.ne = torch.tensor([T // w.m], dtype=torch.int64, device=device)
+        self.O = torch.empty(T, w.H_q, w.c, dtype=torch.bfloat16, device=device)
+        torch.cuda.synchronize(device)
+        log(f"[hca prefill] setup {time.time() - t0:.1f}s: T={T}")
+
+    def step(self):
+        t = self.t
+        E = csa.compress(t["H"], t["W_KV"], t["W_Z"], t["bias"], self.g)
+        win = csa.rmsnorm_rope(t["kv_win"], self.g, pos0=0, pos_step=1)
+        csa.hca_attend(t["q"], t["sink"], E[None], win[None], self.seq, self.pos, self.ne, self.g,
+                       out=self.O)
+
+
 # ---------------------------------------------------------------- timing
 def flush_l2(buf):
     buf.zero_()
@@ -327,8 +353,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill secondary line")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--cpu-queries", type=int, default=32,
-                    help="queries in the CPU-oracle sample (decode workload)")
+                    help="queries in the CPU-oracle sample (decode workload); 0 skips it")
+    ap.add_argument("--workload", default="csa_decode_bf16",
+                    choices=["csa_decode_bf16", "csa_decode_long_mixed"],
+                    help="decode workload of the headline line")
+    ap.add_argument("--batch", type=int, default=0, help="override the decode batch size")
+    ap.add_argument("--prefill-workload", default="csa_prefill_bf16",
+                    choices=["csa_prefill_bf16", "hca_prefill_bf16"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -337,7 +370,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    w = synth.csa_decode_bf16()
+    w = synth.WORKLOADS[args.workload]()
+    if args.batch > 0:
+        w = synth.WORKLOADS[args.workload](B=args.batch)
     config = {"workload": w.name, "batch": w.B, "context": w.L, "entries_per_seq": w.n_entries,
               "m": w.m, "top_k": w.k, "window": w.n_win, "query_heads": w.H_q, "head_dim": w.c,
               "indexer_heads": w.H_I, "indexer_dim": w.c_I, "parallelism": f"dp{args.gpus}",
@@ -384,10 +419,9 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     launches0 = csa.kernel_launches()
     barrier()
-    with Clocks(device.index) as clk:
-        step_ms, idx_ms = time_steps(lambda ev: dec.step(dec.inp, ev), args.steps, args.warmup,
-                                     device, flush,
-                                     extra_events=2)
+    clk = Clocks(device.index).__enter__()
+    step_ms, idx_ms = time_steps(lambda ev: dec.step(dec.inp, ev), args.steps, args.warmup,
+                                 device, flush, extra_events=2)
     launches = csa.kernel_launches() - launches0
     per_step_launches = launches // (args.steps + args.warmup)
     ms = statistics.mean(step_ms)
@@ -395,20 +429,22 @@ def main():
     value = args.gpus * w.B / (ms_max / 1e3)
 
     # end to end through the public API from pinned host memory
-    for _ in range(args.warmup):
-        flush_l2(flush)
-        dec.step_e2e()
-    torch.cuda.synchronize(device)
-    e2e = []
-    for _ in range(args.steps):
-        flush_l2(flush)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        dec.step_e2e()
-        b.record()
-        e2e.append((a, b))
-    torch.cuda.synchronize(device)
-    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e))
+    e2e_ms = None
+    if not args.no_e2e:
+        for _ in range(args.warmup):
+            flush_l2(flush)
+            dec.step_e2e()
+        torch.cuda.synchronize(device)
+        e2e = []
+        for _ in range(args.steps):
+            flush_l2(flush)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            dec.step_e2e()
+            b.record()
+            e2e.append((a, b))
+        torch.cuda.synchronize(device)
+        e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e))
     h2d_bytes, d2h_bytes = dec.h2d_bytes, dec.d2h_bytes
 
     # roofline of the dominant kernel (the indexer)
@@ -433,17 +469,19 @@ def main():
     if not args.no_prefill:
         del dec
         torch.cuda.empty_cache()
-        pw = synth.csa_prefill_bf16()
-        pre = Prefill(pw, device)
+        pw = synth.WORKLOADS[args.prefill_workload]()
+        pre = (Prefill if pw.kind == "csa_prefill" else HcaPrefill)(pw, device)
         pms, _ = time_steps(lambda ev: pre.step(), max(3, args.steps // 4), 3, device, flush)
         pms_max = max_over_ranks(statistics.mean(pms))
-        prefill = {"metric": "CSA prefill tokens/s", "value": args.gpus * pw.T / (pms_max / 1e3),
+        prefill = {"metric": ("CSA" if pw.kind == "csa_prefill" else "HCA") + " prefill tokens/s",
+                   "value": args.gpus * pw.T / (pms_max / 1e3),
                    "unit": "tokens/s", "ms_per_step": pms_max,
                    "config": {"workload": pw.name, "T": pw.T, "d": pw.d, "top_k": pw.k}}
         del pre
 
+    clk.__exit__(None, None, None)
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.cpu_queries > 0:
         nq = max(1, min(args.cpu_queries, w.B))
         qps, el, gen = oracle_decode_sample(w, nq)
         cpu = {"value": qps, "unit": "queries/s", "cores": min(nq, os.cpu_count() or 1),
@@ -458,7 +496,8 @@ def main():
                 "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
                 "roofline": roofline, "cpu_baseline": cpu,
-                "e2e": {"value": args.gpus * w.B / (e2e_ms / 1e3), "unit": "queries/s",
+                "e2e": None if e2e_ms is None else
+                       {"value": args.gpus * w.B / (e2e_ms / 1e3), "unit": "queries/s",
                         "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
                 "gpu_launches": per_step_launches * args.steps,
                 "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
