@@ -57,12 +57,13 @@ _SIGS = {
     "csa_kernel_launches": ([], ctypes.c_uint64),
     "csa_rmsnorm_rope": ([_GP, _I32, _I32, _P, _I64, _P, _I64, _I64, _P, _P, _P, _P], _I32),
     "csa_quantize_mixed": ([_I32, _P, _I64, _P, _P], _I32),
-    "csa_compress_workspace_size": ([_GP, _I64, _I32], _SZ),
+    "csa_compress_workspace_size": ([_GP, _I32, _I64, _I32], _SZ),
     "csa_compress": ([_GP, _I32, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _SZ, _P],
                      _I32),
     "csa_compress_decode_state_floats": ([_GP], _I64),
+    "csa_compress_decode_workspace_size": ([_GP, _I32, _I32, _I32], _SZ),
     "csa_compress_decode": ([_GP, _I32, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P,
-                             _I64, _P], _I32),
+                             _I64, _P, _SZ, _P], _I32),
     "csa_index_topk_workspace_size": ([_I32, _I64, _I32], _SZ),
     "csa_index_topk": ([_GP, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _I32, _I32, _I32,
                         _P, _P, _P, _SZ, _P], _I32),
@@ -174,7 +175,7 @@ def compress(H, W_aKV, W_aZ, bias, g: Geom, W_bKV=None, W_bZ=None, gain=None, ou
     T, d = H.shape
     odt = _dt(H) if out_dtype is None else out_dtype
     E = _rows_out((T // g.m,), g.c, odt, H.device)
-    ws_bytes = load().csa_compress_workspace_size(ctypes.byref(g), T, d)
+    ws_bytes = load().csa_compress_workspace_size(ctypes.byref(g), _dt(H), T, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=H.device)
     _call("csa_compress", ctypes.byref(g), _dt(H), _ptr(H), T, d, _ptr(W_aKV), _ptr(W_bKV),
@@ -190,13 +191,17 @@ def decode_state(B, g: Geom, device="cuda"):
 
 
 def compress_decode(h, pos, W_aKV, W_aZ, bias, state, E_cache, g: Geom, W_bKV=None, W_bZ=None,
-                    gain=None):
+                    gain=None, workspace=None):
     """One decode step of the compressor: h [B, d] at positions pos [B]."""
     _check(h, pos, W_aKV, W_aZ, bias, state, E_cache, W_bKV, W_bZ, gain)
     B, d = h.shape
+    ws_bytes = load().csa_compress_decode_workspace_size(ctypes.byref(g), _dt(h), B, d)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=h.device)
     _call("csa_compress_decode", ctypes.byref(g), _dt(h), _ptr(h), _ptr(pos), B, d, _ptr(W_aKV),
           _ptr(W_bKV), _ptr(W_aZ), _ptr(W_bZ), _ptr(bias), _ptr(gain), _ptr(state),
-          _dt(E_cache), _ptr(E_cache), E_cache.shape[1], _stream(h))
+          _dt(E_cache), _ptr(E_cache), E_cache.shape[1], _ptr(workspace),
+          0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(h))
 
 
 def index_topk(qI, w, KI, seq_of_q, pos, n_entries, k, g: Geom, want_scores=False,

@@ -104,9 +104,9 @@ csa_status csa_quantize_mixed(csa_dtype in_dtype, const void* x, int64_t rows, v
                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
-size_t csa_compress_workspace_size(const csa_geom* g, int64_t T, int d) {
-  (void)d;
-  if (!g || T < 0 || g->c <= 0) return 0;
+size_t csa_compress_workspace_size(const csa_geom* g, csa_dtype dtype, int64_t T, int d) {
+  if (!g || T < 0 || g->c <= 0 || g->m < 1) return 0;
+  if (csa::proj_tc_supported(*g, dtype, d)) return csa::proj_pool_workspace(*g, T);
   const int nW = g->overlap ? 4 : 2;
   return (size_t)T * nW * g->c * sizeof(float);
 }
@@ -124,12 +124,19 @@ csa_status csa_compress(const csa_geom* g, csa_dtype dtype, const void* H, int64
   for (const void* p : ptrs)
     if (!aligned16(p)) return CSA_ERR_INVALID_ARG;
   if (T / g->m == 0) return CSA_OK;
-  if (!workspace || ws_bytes < csa_compress_workspace_size(g, T, d)) return CSA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < csa_compress_workspace_size(g, dtype, T, d)) return CSA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* P = reinterpret_cast<float*>(workspace);
   const int nW = g->overlap ? 4 : 2;
   // projections in the order [C^a | Z^a | C^b | Z^b]
   const void* W[4] = {W_aKV, W_aZ, W_bKV, W_bZ};
+  if (csa::proj_tc_supported(*g, dtype, d)) {
+    // tensor-core projection with the pool fused, then RMSNorm + RoPE at i*m
+    cudaError_t e = csa::launch_compress_tc(*g, H, T, d, W, bias, P, s);
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
+    return cuda_status(csa::launch_rmsnorm_rope(*g, CSA_F32, out_dtype, P, T / g->m, nullptr, 0,
+                                                g->m, gain, E_out, nullptr, s));
+  }
   const int64_t Tc = (T / g->m) * g->m;  // tokens after the last complete block are unused
   cudaError_t e = csa::launch_proj_simt(dtype, H, Tc, d, g->c, nW, W, P, s);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
@@ -143,33 +150,47 @@ int64_t csa_compress_decode_state_floats(const csa_geom* g) {
   return (int64_t)nslot * g->m * nW * g->c;
 }
 
+size_t csa_compress_decode_workspace_size(const csa_geom* g, csa_dtype dtype, int B, int d) {
+  if (!g || B <= 0 || d < 1 || g->c <= 0) return 0;
+  return csa::proj_decode_supported(*g, dtype, d) ? csa::proj_decode_workspace(*g, B, d) : 0;
+}
+
 csa_status csa_compress_decode(const csa_geom* g, csa_dtype dtype, const void* h,
                                const int64_t* pos, int B, int d, const void* W_aKV,
                                const void* W_bKV, const void* W_aZ, const void* W_bZ,
                                const float* bias, const float* gain, float* state,
-                               csa_dtype out_dtype, void* E_cache, int64_t ldE,
-                               csa_stream_t stream) {
+                               csa_dtype out_dtype, void* E_cache, int64_t ldE, void* workspace,
+                               size_t ws_bytes, csa_stream_t stream) {
   if (!geom_ok(g) || !io_dtype_ok(dtype) || !out_dtype_ok(g, out_dtype)) return CSA_ERR_INVALID_ARG;
   if (B < 0 || d < 1 || ldE < 0) return CSA_ERR_INVALID_ARG;
   if (B == 0) return CSA_OK;
   if (!h || !pos || !W_aKV || !W_aZ || !bias || !state || !E_cache) return CSA_ERR_INVALID_ARG;
   if (g->overlap ? (!W_bKV || !W_bZ) : (W_bKV || W_bZ)) return CSA_ERR_INVALID_ARG;
-  const void* ptrs[] = {h, pos, W_aKV, W_bKV, W_aZ, W_bZ, bias, gain, state, E_cache};
+  const void* ptrs[] = {h, pos, W_aKV, W_bKV, W_aZ, W_bZ, bias, gain, state, E_cache, workspace};
   for (const void* p : ptrs)
     if (!aligned16(p)) return CSA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int nW = g->overlap ? 4 : 2;
   const void* W[4] = {W_aKV, W_aZ, W_bKV, W_bZ};
-  cudaError_t e = csa::launch_decode_proj(*g, dtype, h, pos, B, d, W, nW, state, s);
+  const size_t need = csa_compress_decode_workspace_size(g, dtype, B, d);
+  if (need > 0 && (!workspace || ws_bytes < need)) return CSA_ERR_INVALID_ARG;
+  cudaError_t e = need > 0 ? csa::launch_decode_proj_tc(*g, h, pos, B, d, W,
+                                                        reinterpret_cast<float*>(workspace), state, s)
+                           : csa::launch_decode_proj(*g, dtype, h, pos, B, d, W, nW, state, s);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   return cuda_status(csa::launch_decode_pool(*g, pos, B, bias, gain, state, out_dtype, E_cache,
                                              ldE, s));
 }
 
+// workspace of csa_index_topk: FP32 scores [Q, ldK], then the top-k
+// chunk candidates (256-byte aligned)
+static size_t scores_bytes(int Q, int64_t ldK) {
+  return ((size_t)Q * (size_t)ldK * sizeof(float) + 255) / 256 * 256;
+}
+
 size_t csa_index_topk_workspace_size(int Q, int64_t ldK, int k) {
-  (void)k;
-  if (Q < 0 || ldK < 0) return 0;
-  return (size_t)Q * (size_t)ldK * sizeof(float);
+  if (Q < 0 || ldK < 0 || k < 1) return 0;
+  return scores_bytes(Q, ldK) + csa::topk_workspace(Q, ldK, k);
 }
 
 csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, const float* w,
@@ -180,6 +201,7 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
   if (!geom_ok(g) || !io_dtype_ok(dtype)) return CSA_ERR_INVALID_ARG;
   if (Q < 0 || H_I < 1 || H_I > 128 || c_I < 16 || (c_I % 16) != 0 || c_I > 256) return CSA_ERR_INVALID_ARG;
   if (k < 1 || k > CSA_MAX_TOPK || ldK < 0 || nseq < 0) return CSA_ERR_INVALID_ARG;
+  if (!csa::topk_supported(ldK, k)) return CSA_ERR_UNSUPPORTED;
   if (Q == 0) return CSA_OK;
   if (!qI || !w || !KI || !seq_of_q || !pos || !n_entries || !idx_out) return CSA_ERR_INVALID_ARG;
   const void* ptrs[] = {qI, w, KI, seq_of_q, pos, n_entries, idx_out, scores_dbg, workspace};
@@ -198,8 +220,9 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
                                                         s);
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
-  return cuda_status(csa::launch_topk_from_scores(*g, scores, ldK, nseq, seq_of_q, pos, n_entries,
-                                                  Q, k, idx_out, scores_dbg, ldK, s));
+  void* cand = reinterpret_cast<uint8_t*>(workspace) + scores_bytes(Q, ldK);
+  return cuda_status(csa::launch_topk(*g, scores, ldK, nseq, seq_of_q, pos, n_entries, Q, k,
+                                      idx_out, scores_dbg, ldK, cand, s));
 }
 
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win) {

@@ -40,10 +40,13 @@ cudaError_t launch_index_scores_simt(const csa_geom& g, int dt, const void* qI, 
                                      const int32_t* seq_of_q,
                                      const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
                                      int c_I, float* scores, int64_t ld_scores, cudaStream_t s);
-cudaError_t launch_topk_from_scores(const csa_geom& g, const float* scores, int64_t ld_scores,
-                                    int nseq, const int32_t* seq_of_q, const int64_t* pos,
-                                    const int64_t* n_entries, int Q, int k, int32_t* idx_out,
-                                    float* scores_dbg, int64_t ld_dbg, cudaStream_t s);
+// Exact top-k of per-query scores [Q, ld_scores] (topk.cu).
+bool topk_supported(int64_t ld_scores, int k);
+size_t topk_workspace(int Q, int64_t ld_scores, int k);
+cudaError_t launch_topk(const csa_geom& g, const float* scores, int64_t ld_scores, int nseq,
+                        const int32_t* seq_of_q, const int64_t* pos, const int64_t* n_entries,
+                        int Q, int k, int32_t* idx_out, float* scores_dbg, int64_t ld_dbg,
+                        void* cand_ws, cudaStream_t s);
 // ---- tensor-core kernels (tc_*.cu) ----
 bool index_tc_supported(int dt, int H_I, int c_I);
 cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const float* w,
@@ -51,6 +54,18 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
                                    const int32_t* seq_of_q, const int64_t* pos,
                                    const int64_t* n_entries, int Q, int H_I, int c_I,
                                    float* scores, int64_t ld_scores, cudaStream_t s);
+bool proj_tc_supported(const csa_geom& g, int dt, int d);
+bool proj_decode_supported(const csa_geom& g, int dt, int d);
+size_t proj_pool_workspace(const csa_geom& g, int64_t T);
+size_t proj_decode_workspace(const csa_geom& g, int B, int d);
+// pooled [T/m, c] FP32 (before RMSNorm/RoPE) of a prefill sequence
+cudaError_t launch_compress_tc(const csa_geom& g, const void* H, int64_t T, int d,
+                               const void* const* W, const float* bias, float* pooled,
+                               cudaStream_t s);
+// projections of one new token per sequence into the decode state
+cudaError_t launch_decode_proj_tc(const csa_geom& g, const void* h, const int64_t* pos, int B,
+                                  int d, const void* const* W, float* part, float* state,
+                                  cudaStream_t s);
 bool attend_tc_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_dims);
 size_t attend_tc_workspace(int Q, int64_t max_slots);
 cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,

@@ -65,124 +65,6 @@ __global__ void __launch_bounds__(128) index_scores_simt_kernel(
   scores[(int64_t)q * ld_scores + s] = I;
 }
 
-// ---------------------------------------------------------------------------
-// Top-k by radix select on order-preserving 32-bit keys, one block per
-// query; ties at the threshold keep the lowest indices; output ascending.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-constexpr int kTopkThreads = 1024;
-
-template <int NT>
-__device__ int block_exclusive_scan(int v, int* sh, int* total) {
-  // sh: NT/32 ints scratch
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh[wid] = x;
-  __syncthreads();
-  if (wid == 0) {
-    int s = lane < NT / 32 ? sh[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < NT / 32) sh[lane] = s;
-  }
-  __syncthreads();
-  int base = wid > 0 ? sh[wid - 1] : 0;
-  *total = sh[NT / 32 - 1];
-  __syncthreads();
-  return base + x - v;
-}
-
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(
-    csa_geom g, const float* __restrict__ scores, int64_t ld_scores,
-    int nseq, const int32_t* __restrict__ seq_of_q, const int64_t* __restrict__ pos,
-    const int64_t* __restrict__ n_entries, int k, int32_t* __restrict__ idx_out,
-    float* __restrict__ scores_dbg, int64_t ld_dbg) {
-  __shared__ int hist[256];
-  __shared__ int scan_sh[kTopkThreads / 32];
-  __shared__ uint32_t sh_prefix;
-  __shared__ int sh_remaining;
-  const int q = blockIdx.x;
-  const int b = seq_of_q[q];
-  const int64_t nv =
-      (b < 0 || b >= nseq) ? 0 : n_visible(pos[q], g.m, g.vis_offset, min(n_entries[b], ld_scores));
-  const float* sc = scores + (int64_t)q * ld_scores;
-  int32_t* out = idx_out + (int64_t)q * k;
-  if (scores_dbg)
-    for (int64_t s = threadIdx.x; s < nv; s += kTopkThreads) scores_dbg[(int64_t)q * ld_dbg + s] = sc[s];
-  if (nv <= k) {
-    for (int64_t j = threadIdx.x; j < k; j += kTopkThreads) out[j] = j < nv ? (int32_t)j : -1;
-    return;
-  }
-  // radix select of the k-th largest key, 8 bits per pass from the top
-  uint32_t prefix = 0, mask = 0;
-  int remaining = k;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int e = threadIdx.x; e < 256; e += kTopkThreads) hist[e] = 0;
-    __syncthreads();
-    for (int64_t s = threadIdx.x; s < nv; s += kTopkThreads) {
-      uint32_t key = order_key(sc[s]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int cum = 0, dsel = 0;
-      for (int dg = 255; dg >= 0; --dg) {
-        if (cum + hist[dg] >= remaining) {
-          dsel = dg;
-          break;
-        }
-        cum += hist[dg];
-      }
-      sh_prefix = prefix | ((uint32_t)dsel << shift);
-      sh_remaining = remaining - cum;
-    }
-    __syncthreads();
-    prefix = sh_prefix;
-    remaining = sh_remaining;
-    mask |= 255u << shift;
-    __syncthreads();
-  }
-  // prefix = threshold key; `remaining` ties at the threshold are kept
-  const uint32_t thr = prefix;
-  const int64_t per = (nv + kTopkThreads - 1) / kTopkThreads;
-  const int64_t a0 = threadIdx.x * per;
-  const int64_t a1 = min(nv, a0 + per);
-  int nsel = 0, ntie = 0;
-  for (int64_t s = a0; s < a1; ++s) {
-    uint32_t key = order_key(sc[s]);
-    nsel += key > thr;
-    ntie += key == thr;
-  }
-  int tot;
-  const int tie_base = block_exclusive_scan<kTopkThreads>(ntie, scan_sh, &tot);
-  int take_ties = remaining - tie_base;
-  take_ties = take_ties < 0 ? 0 : (take_ties > ntie ? ntie : take_ties);
-  const int out_base = block_exclusive_scan<kTopkThreads>(nsel + take_ties, scan_sh, &tot);
-  int o = out_base, tl = 0;
-  for (int64_t s = a0; s < a1; ++s) {
-    uint32_t key = order_key(sc[s]);
-    bool keep = key > thr;
-    if (key == thr) {
-      keep = tl < take_ties;
-      ++tl;
-    }
-    if (keep) out[o++] = (int32_t)s;
-  }
-  // k_eff = k here (nv > k)
-}
-
 }  // namespace
 
 template <typename Tin, int HMAX>
@@ -221,17 +103,6 @@ cudaError_t launch_index_scores_simt(const csa_geom& g, int dt, const void* qI, 
   CSA_IDX_CASE(128)
 #undef CSA_IDX_CASE
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_topk_from_scores(const csa_geom& g, const float* scores, int64_t ld_scores,
-                                    int nseq, const int32_t* seq_of_q, const int64_t* pos,
-                                    const int64_t* n_entries, int Q, int k, int32_t* idx_out,
-                                    float* scores_dbg, int64_t ld_dbg, cudaStream_t s) {
-  if (Q == 0) return cudaSuccess;
-  count_launches();
-  topk_kernel<<<Q, kTopkThreads, 0, s>>>(g, scores, ld_scores, nseq, seq_of_q, pos, n_entries, k,
-                                         idx_out, scores_dbg, ld_dbg);
-  return cudaGetLastError();
 }
 
 }  // namespace csa

@@ -53,7 +53,9 @@ constexpr int kOffRed = kOffP + 16384;             // 4 x 64 floats
 constexpr int kOffRef = kOffRed + 4 * kHeads * 4;  // 64 floats (log2 units)
 constexpr int kOffAlpha = kOffRef + kHeads * 4;    // 64 floats
 constexpr int kOffMisc = kOffAlpha + kHeads * 4;   // barriers, tmem slot, flags
-constexpr int kOffList = kOffMisc + 64;            // compacted entry list
+constexpr int kOffRope = kOffMisc + 64;            // 32 x (cos, sin) at the query position
+constexpr int kOffInv = kOffRope + 32 * 8;         // 64 floats: 1 / denominator per head
+constexpr int kOffList = kOffInv + kHeads * 4;     // compacted entry list
 constexpr int kSmemFixed = kOffList + 1024;        // + alignment slack
 
 struct Params {
@@ -101,6 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kOffMisc + 16);
   int* flags = reinterpret_cast<int*>(sm + kOffMisc + 32);  // [0] abort, [1] rescale, [2] nvalid
   int32_t* list = reinterpret_cast<int32_t*>(sm + kOffList);
+  float2* rope = reinterpret_cast<float2*>(sm + kOffRope);
+  float* inv_den = reinterpret_cast<float*>(sm + kOffInv);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qi = blockIdx.y;
@@ -119,7 +123,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
     flags[1] = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 8) tc::tmem_alloc(tc::smem_u32(tslot), kTmemCols);
+  if (warp == 8) {
+    tc::tmem_alloc(tc::smem_u32(tslot), kTmemCols);
+    // cos/sin of the query position for each rotated pair (FP64 angles)
+    if (lane < P.r / 2) {
+      float cs, sn;
+      rope_cs(p, lane, P.r, P.base, &cs, &sn);
+      rope[lane] = make_float2(cs, sn);
+    }
+  }
   const int64_t ldE = P.ldE;
   int64_t nsel = 0;
   if (valid_seq) {
@@ -151,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       }
     }
   }
+  __syncthreads();  // RoPE table ready
   // ---- q-hat = RoPE_p(RMSNorm(q_h) * gain) in BF16, K-major swizzled ----
   if (valid_seq && warp < 8) {
     for (int h = warp; h < kHeads; h += 8) {
@@ -179,10 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
         float a = v[i] * inv * (P.q_gain ? P.q_gain[d] : 1.f);
         float bb = v[i + 1] * inv * (P.q_gain ? P.q_gain[d + 1] : 1.f);
         if (d >= kDim - P.r) {
-          float cs, sn;
-          rope_cs(p, (d - (kDim - P.r)) >> 1, P.r, P.base, &cs, &sn);
-          const float a2 = a * cs - bb * sn;
-          bb = a * sn + bb * cs;
+          const float2 t = rope[(d - (kDim - P.r)) >> 1];
+          const float a2 = a * t.x - bb * t.y;
+          bb = a * t.y + bb * t.x;
           a = a2;
         }
         v[i] = a;
@@ -398,13 +410,23 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       if (lane == 0) red[quad * kHeads + h] = v;
     }
     tc::named_bar(1, 128);
-    const int dim_in_blk = quad * 32 + lane;
     const bool split_mode = P.tiles_per_split > 0;
+    if (warp == 4 || warp == 5) {
+      const int h = (warp - 4) * 32 + lane;
+      const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
+      inv_den[h] = 1.f / (l + exp2f(P.sink[h] * kLog2e - ref2[h]));
+    }
+    tc::named_bar(1, 128);
+    const int dim_in_blk = quad * 32 + lane;
     for (int blk = 0; blk < 4; ++blk) {
       const int d = blk * 128 + dim_in_blk;
       float cs = 1.f, sn = 0.f;
       const bool rot = d >= kDim - P.r;
-      if (rot && !split_mode) rope_cs(p, (d - (kDim - P.r)) >> 1, P.r, P.base, &cs, &sn);
+      if (rot) {
+        const float2 t = rope[(d - (kDim - P.r)) >> 1];
+        cs = t.x;
+        sn = t.y;
+      }
       for (int c0 = 0; c0 < kHeads; c0 += 32) {
         float o[32];
         if (have) {
@@ -416,12 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int h = c0 + i;
-          const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
           if (split_mode) {
             P.part_O[(((int64_t)qi * P.max_splits + split) * kHeads + h) * kDim + d] = have ? o[i] : 0.f;
           } else {
-            const float den = l + exp2f(P.sink[h] * kLog2e - ref2[h]);
-            float val = valid_seq ? o[i] / den : 0.f;
+            float val = valid_seq ? o[i] * inv_den[h] : 0.f;
             if (rot) {
               // pair (d, d^1) sits in the neighbouring lane; rotate by -p
               const float other = __shfl_xor_sync(0xffffffffu, val, 1);
@@ -493,7 +513,7 @@ int choose_tiles_per_split(int Q, int64_t max_slots) {
 
 bool attend_tc_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_dims) {
   return q_dt == CSA_BF16 && (kv_dt == CSA_BF16 || kv_dt == CSA_FP8_MIXED) && c == kDim &&
-         H_q == kHeads && k <= CSA_MAX_TOPK && rope_dims % 32 == 0;
+         H_q == kHeads && k <= CSA_MAX_TOPK && rope_dims % 32 == 0 && rope_dims <= 64;
 }
 
 size_t attend_tc_workspace(int Q, int64_t max_slots) {

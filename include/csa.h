@@ -161,9 +161,9 @@ csa_status csa_quantize_mixed(csa_dtype in_dtype, const void* x, int64_t rows, v
  *   gain  [c] FP32, NULL = ones
  *   E_out [floor(T/m), c] out_dtype (F32, BF16 or CSA_FP8_MIXED rows)
  * Tokens after the last complete block are not pooled.
- * workspace: csa_compress_workspace_size() bytes.
+ * workspace: csa_compress_workspace_size() bytes for the same dtype.
  * --------------------------------------------------------------------- */
-size_t csa_compress_workspace_size(const csa_geom* g, int64_t T, int d);
+size_t csa_compress_workspace_size(const csa_geom* g, csa_dtype dtype, int64_t T, int d);
 csa_status csa_compress(const csa_geom* g, csa_dtype dtype, const void* H, int64_t T, int d,
                         const void* W_aKV, const void* W_bKV, const void* W_aZ,
                         const void* W_bZ, const float* bias, const float* gain,
@@ -186,14 +186,17 @@ csa_status csa_compress(const csa_geom* g, csa_dtype dtype, const void* H, int64
  * pooled, normalised, rotated and written to E_cache[b, i] (i < ldE is the
  * caller's responsibility; entries i >= ldE are skipped).
  * Tokens must arrive in position order per sequence.
+ * workspace: csa_compress_decode_workspace_size() bytes (split-K partial
+ * projections of the batch).
  * --------------------------------------------------------------------- */
 int64_t csa_compress_decode_state_floats(const csa_geom* g);
+size_t csa_compress_decode_workspace_size(const csa_geom* g, csa_dtype dtype, int B, int d);
 csa_status csa_compress_decode(const csa_geom* g, csa_dtype dtype, const void* h,
                                const int64_t* pos, int B, int d, const void* W_aKV,
                                const void* W_bKV, const void* W_aZ, const void* W_bZ,
                                const float* bias, const float* gain, float* state,
-                               csa_dtype out_dtype, void* E_cache, int64_t ldE,
-                               csa_stream_t stream);
+                               csa_dtype out_dtype, void* E_cache, int64_t ldE, void* workspace,
+                               size_t ws_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------
  * csa_index_topk - lightning indexer and top-k selection.

@@ -45,7 +45,8 @@ def test_status_strings(lib):
 
 def test_workspace_queries(lib):
     g = csa.geom()
-    assert lib.csa_compress_workspace_size(ctypes.byref(g), 8192, 4096) >= 8192 * 4 * 512 * 4
+    assert lib.csa_compress_workspace_size(ctypes.byref(g), 0, 8192, 4096) >= 8192 * 4 * 512 * 4
+    assert lib.csa_compress_workspace_size(ctypes.byref(g), 1, 8192, 4096) >= 2048 * 512 * 4
     assert lib.csa_index_topk_workspace_size(32, 32768, 1024) >= 0
     assert lib.csa_compress_decode_state_floats(ctypes.byref(g)) == 2 * 4 * 4 * 512
     gh = csa.geom(m=128, overlap=0)

@@ -242,6 +242,17 @@ def test_index_topk_grouped_queries(orc, HI, cI):
         assert max_abs(sc[q, :nv], ref["scores"][q, :nv]) <= 2.0 ** -14 * ref["amag"][q] + 1e-6
 
 
+@pytest.mark.parametrize("k", [1024, 300])
+def test_index_topk_many_entries_bit_exact(orc, k):
+    """More visible entries than one selection block holds: chunk top-k
+    candidates are merged; integer inputs make the result exact."""
+    qI, w, KI, seq, pos, ne = _index_inputs(6, 16, 64, 2, 21000, "bf16", integer=True, seed=8)
+    pos[:] = [4 * 21000, 4 * 21000 + 7, 4 * 9000, 4 * 16384 - 1, 4 * 16384, 5]
+    idx = _run_index(qI, w, KI, seq, pos, ne, k, "bf16").cpu().numpy()
+    want = orc.index_topk(qI, w, KI, seq, pos, ne, m=4, k=k)["idx"]
+    np.testing.assert_array_equal(idx, want)
+
+
 def test_index_topk_no_visible_entries(orc):
     qI, w, KI, seq, pos, ne = _index_inputs(8, 4, 32, 1, 50, "f32", seed=5)
     pos[:] = [0, 1, 2, 3, 4, 5, 6, 7]
