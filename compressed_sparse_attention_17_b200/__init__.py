@@ -24,7 +24,7 @@ LIB_PATH = Path(__file__).resolve().parent / "libcsa.so"
 MIXED_ROW_BYTES = 592
 CSA_F32, CSA_BF16, CSA_FP8_MIXED = 0, 1, 2
 _STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CUDA",
-           4: "CSA_ERR_TIMEOUT"}
+           4: "CSA_ERR_TIMEOUT", 5: "CSA_ERR_TOO_LARGE"}
 
 
 class CsaError(RuntimeError):
@@ -67,6 +67,8 @@ _SIGS = {
     "csa_index_topk_workspace_size": ([_I32, _I64, _I32], _SZ),
     "csa_index_topk": ([_GP, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _I32, _I32, _I32,
                         _P, _P, _P, _SZ, _P], _I32),
+    "csa_index_topk_noalloc": ([_GP, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _I32, _I32,
+                                _I32, _P, _P, _P], _I32),
     "csa_attend_workspace_size": ([_I32, _I32, _I32, _I32, _I32], _SZ),
     "csa_attend": ([_GP, _I32, _I32, _P, _P, _P, _P, _I64, _I32, _P, _P, _I32, _P, _I64, _P, _P,
                     _I32, _I32, _P, _P, _SZ, _P], _I32),

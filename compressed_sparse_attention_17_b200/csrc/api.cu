@@ -59,6 +59,7 @@ const char* csa_status_string(csa_status s) {
     case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
     case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
     case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT";
+    case CSA_ERR_TOO_LARGE: return "CSA_ERR_TOO_LARGE";
   }
   return "CSA_ERR_UNKNOWN";
 }

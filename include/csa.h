@@ -67,7 +67,9 @@ typedef enum {
   CSA_ERR_INVALID_ARG = 1,
   CSA_ERR_UNSUPPORTED = 2,
   CSA_ERR_CUDA = 3,
-  CSA_ERR_TIMEOUT = 4
+  CSA_ERR_TIMEOUT = 4,
+  CSA_ERR_TOO_LARGE = 5 /* the call needs more scratch than the fixed buffer
+                           of csa_index_topk_noalloc() holds */
 } csa_status;
 
 typedef enum {
@@ -224,6 +226,35 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
                           const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
                           int c_I, int k, int32_t* idx_out, float* scores_dbg,
                           void* workspace, size_t ws_bytes, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------
+ * csa_index_topk_noalloc - csa_index_topk without a caller workspace.
+ * (An interface addition of this library; the pages have no counterpart.)
+ * For callers that cannot allocate device memory around the call - code
+ * running inside a memory arena that forbids outside allocations, or a
+ * serving loop that must not allocate - the scores and top-k candidates
+ * live in one fixed device buffer of CSA_NOALLOC_SCRATCH_BYTES compiled into
+ * the library (every GPU that loads the library holds it until the process
+ * exits). Arguments and results are those of csa_index_topk.
+ *   - Returns CSA_ERR_TOO_LARGE, launching nothing, when
+ *     csa_index_topk_workspace_size(Q, ldK, k) exceeds the buffer.
+ *   - The first call on each device looks up the buffer's device address
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *     routine.
+ *   - Every call shares the one buffer, which keeps the last call's
+ *     contents; nothing in it needs to start at zero (each value read is
+ *     written earlier in the same call). Calls that overlap on the GPU
+ *     (other streams, other host threads) race on the buffer: serialise
+ *     them.
+ * --------------------------------------------------------------------- */
+#define CSA_NOALLOC_SCRATCH_BYTES (8u << 20)
+csa_status csa_index_topk_noalloc(const csa_geom* g, csa_dtype dtype, const void* qI,
+                                  const float* w, const void* KI, int64_t ldK, int nseq,
+                                  const int32_t* seq_of_q, const int64_t* pos,
+                                  const int64_t* n_entries, int Q, int H_I, int c_I, int k,
+                                  int32_t* idx_out, float* scores_dbg, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------
  * csa_attend - shared-KV multi-query core attention over the selected
