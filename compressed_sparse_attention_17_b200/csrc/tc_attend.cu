@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       const int64_t slot = t * kTile + key;
       const bool kvalid = slot < nslots;
       float s[kHeads];
-      const bool ok = tc::mbar_wait(s_bar, phase, P.err);
+      const bool ok = tc::mbar_wait_warp(s_bar, phase, P.err);
       if (!ok) flags[0] = 1;
       tc::tc_fence_after();
       tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + kColS, s);
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       }
       tc::mma_commit(o_bar);
     }
-    if (!tc::mbar_wait(o_bar, phase, P.err)) flags[0] = 1;
+    if (!tc::mbar_wait_warp(o_bar, phase, P.err)) flags[0] = 1;
     tc::tc_fence_after();
     phase ^= 1u;
     __syncthreads();

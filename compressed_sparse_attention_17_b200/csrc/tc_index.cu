@@ -15,6 +15,8 @@
 //
 // Warp roles (192 threads): warp 0 issues the TMA loads, warp 1 owns the
 // TMEM allocation and issues the MMAs, warps 2-5 run the epilogue.
+#include <algorithm>
+
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       } else if (warp >= 2) {
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
-        if (tc::mbar_wait(mma_bar, phase, P.err)) {
+        if (tc::mbar_wait_warp(mma_bar, phase, P.err)) {
           tc::tc_fence_after();
           const int64_t s = s0 + row;
           for (int j = j0; j < j1; ++j) {
@@ -161,6 +163,247 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 1) tc::tmem_dealloc(tmem, P.tmem_cols);
 }
 
+// ---------------------------------------------------------------------------
+// Persistent, pipelined variant for few queries (decode): every CTA takes a
+// balanced contiguous range of (query, 128-entry tile) units, which may span
+// query boundaries. Warp 0 streams the key tiles through a ring of shared-
+// memory stages (TMA, evict-first L2 policy: keys are read once) and loads
+// a query's qI into one of two slots when the query changes; warp 1 issues
+// the MMAs into one of two TMEM accumulators; warps 2-5 reduce the previous
+// accumulator while the next tile is multiplied and later tiles load.
+// ---------------------------------------------------------------------------
+constexpr int kDecMaxQ = 1024;
+
+struct DecParams {
+  int Q, H_I, c_I, nseq, stages;
+  int64_t ldK;
+  int m, vis_offset;
+  const int32_t* seq_of_q;
+  const int64_t* pos;
+  const int64_t* n_entries;
+  const float* w;
+  float* scores;
+  int64_t ld_scores;
+  int* err;
+  uint32_t tmem_cols;
+};
+
+__device__ __forceinline__ int64_t dec_nvis(const DecParams& P, int q) {
+  const int b = P.seq_of_q[q];
+  if (b < 0 || b >= P.nseq) return 0;
+  return n_visible(P.pos[q], P.m, P.vis_offset, min(P.n_entries[b], P.ldK));
+}
+
+// Walks units [u0, u1) in order; prefix[q] = first unit of query q.
+struct UnitWalk {
+  const int* prefix;
+  int Q;
+  int q;
+  int64_t t;
+  __device__ void start(const int* pre, int nq, int u0) {
+    prefix = pre;
+    Q = nq;
+    int lo = 0, hi = nq - 1;  // largest q with prefix[q] <= u0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= u0) lo = mid;
+      else hi = mid - 1;
+    }
+    q = lo;
+    t = u0 - prefix[q];
+    while (q < Q - 1 && t >= prefix[q + 1] - prefix[q]) {
+      t -= prefix[q + 1] - prefix[q];
+      ++q;
+    }
+  }
+  __device__ void next() {
+    ++t;
+    while (q < Q - 1 && t >= prefix[q + 1] - prefix[q]) {
+      t = 0;
+      ++q;
+    }
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    index_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                        DecParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int KCH = P.c_I / 64;
+  const int S = P.stages;
+  const int bytesA = KCH * kChunkBytesA;
+  const int bytesB = KCH * P.H_I * 128;
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * bytesA;
+  float* wsm = reinterpret_cast<float*>(sB + 2 * bytesB);
+  int* prefix = reinterpret_cast<int*>(wsm + 128);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + ((P.Q + 2 + 1) & ~1));
+  // bars: Afull[S], Aempty[S], Bfull[2], Bempty[2], accfull[2], accempty[2]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
+  __shared__ int scan_tmp[kThreads / 32];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- units per query and their prefix (every CTA computes it) ----
+  int carry = 0;
+  for (int base = 0; base < P.Q; base += kThreads) {
+    const int q = base + threadIdx.x;
+    const int nt = q < P.Q ? (int)((dec_nvis(P, q) + kTileM - 1) / kTileM) : 0;
+    int x = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) scan_tmp[warp] = x;
+    __syncthreads();
+    int wbase = 0, tot = 0;
+    for (int i = 0; i < kThreads / 32; ++i) {
+      wbase += i < warp ? scan_tmp[i] : 0;
+      tot += scan_tmp[i];
+    }
+    if (q < P.Q) prefix[q] = carry + wbase + x - nt;
+    carry += tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) prefix[P.Q] = carry;
+  __syncthreads();
+  const int U = prefix[P.Q];
+  const int u0 = (int)((int64_t)blockIdx.x * U / gridDim.x);
+  const int u1 = (int)((int64_t)(blockIdx.x + 1) * U / gridDim.x);
+  if (u0 >= u1) return;  // same decision in every thread of the CTA
+
+  auto afull = [&](int s) { return tc::smem_u32(&bars[s]); };
+  auto aempty = [&](int s) { return tc::smem_u32(&bars[S + s]); };
+  auto bfull = [&](int s) { return tc::smem_u32(&bars[2 * S + s]); };
+  auto bempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 2 + s]); };
+  auto accfull = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + s]); };
+  auto accempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 6 + s]); };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(afull(s), 1);
+      tc::mbar_init(aempty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(bfull(s), 1);
+      tc::mbar_init(bempty(s), 1);
+      tc::mbar_init(accfull(s), 1);
+      tc::mbar_init(accempty(s), 4);
+    }
+    tc::fence_barrier_init();
+    tc::prefetch_tmap(&tmK);
+    tc::prefetch_tmap(&tmQ);
+  }
+  if (warp == 1) tc::tmem_alloc(tc::smem_u32(tslot), P.tmem_cols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const int nunits = u1 - u0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer ----
+      const uint64_t pol = tc::l2_policy_evict_first();
+      UnitWalk wk;
+      wk.start(prefix, P.Q, u0);
+      int last_q = -1, gc = -1;
+      for (int i = 0; i < nunits; ++i, wk.next()) {
+        const int q = wk.q;
+        if (q != last_q) {
+          ++gc;
+          const int bs = gc & 1;
+          if (gc >= 2 && !tc::mbar_wait(bempty(bs), ((gc >> 1) - 1) & 1, P.err)) break;
+          tc::mbar_arrive_expect_tx(bfull(bs), (uint32_t)bytesB);
+          for (int ch = 0; ch < KCH; ++ch)
+            tc::tma_load_2d(tc::smem_u32(sB + bs * bytesB + ch * P.H_I * 128), &tmQ, ch * 64,
+                            q * P.H_I, bfull(bs));
+          last_q = q;
+        }
+        const int s = i % S;
+        if (i >= S && !tc::mbar_wait(aempty(s), ((i / S) - 1) & 1, P.err)) break;
+        tc::mbar_arrive_expect_tx(afull(s), (uint32_t)bytesA);
+        const int32_t y = (int32_t)((int64_t)P.seq_of_q[q] * P.ldK + wk.t * kTileM);
+        for (int ch = 0; ch < KCH; ++ch)
+          tc::tma_load_2d_hint(tc::smem_u32(sA + s * bytesA + ch * kChunkBytesA), &tmK, ch * 64, y,
+                               afull(s), pol);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      const uint32_t idesc = tc::idesc_bf16_f32(kTileM, P.H_I);
+      UnitWalk wk;
+      wk.start(prefix, P.Q, u0);
+      int last_q = -1, gc = -1;
+      for (int i = 0; i < nunits; ++i, wk.next()) {
+        const int q = wk.q;
+        if (q != last_q) {
+          if (gc >= 0) tc::mma_commit(bempty(gc & 1));  // previous query's qI slot is free
+          ++gc;
+          if (!tc::mbar_wait(bfull(gc & 1), (gc >> 1) & 1, P.err)) break;
+          last_q = q;
+        }
+        const int s = i % S, a = i & 1;
+        if (!tc::mbar_wait(afull(s), (i / S) & 1, P.err)) break;
+        if (i >= 2 && !tc::mbar_wait(accempty(a), ((i >> 1) - 1) & 1, P.err)) break;
+        tc::tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(a * P.H_I);
+        for (int kk = 0; kk < KCH * 4; ++kk) {
+          const int ch = kk >> 2;
+          const uint32_t off = (uint32_t)(kk & 3) * 32;
+          tc::mma_bf16(d, tc::sdesc_kmajor_sw128(tc::smem_u32(sA + s * bytesA + ch * kChunkBytesA) + off),
+                       tc::sdesc_kmajor_sw128(tc::smem_u32(sB + (gc & 1) * bytesB + ch * P.H_I * 128) + off),
+                       idesc, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(aempty(s));
+        tc::mma_commit(accfull(a));
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: one entry per thread ----
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    UnitWalk wk;
+    wk.start(prefix, P.Q, u0);
+    int last_q = -1;
+    int64_t nv = 0;
+    float* out = nullptr;
+    const float* wq = nullptr;
+    for (int i = 0; i < nunits; ++i, wk.next()) {
+      const int q = wk.q;
+      if (q != last_q) {
+        nv = dec_nvis(P, q);
+        out = P.scores + (int64_t)q * P.ld_scores;
+        wq = P.w + (int64_t)q * P.H_I;
+        last_q = q;
+      }
+      const int a = i & 1;
+      if (!tc::mbar_wait_warp(accfull(a), (i >> 1) & 1, P.err)) break;
+      tc::tc_fence_after();
+      float acc = 0.f;
+      for (int h0 = 0; h0 < P.H_I; h0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * P.H_I + h0), v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc = fmaf(__ldg(wq + h0 + j), fmaxf(v[j], 0.f), acc);
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(accempty(a));
+      const int64_t sidx = wk.t * kTileM + row;
+      if (sidx < nv) out[sidx] = acc;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, P.tmem_cols);
+}
+
 }  // namespace
 
 bool index_tc_supported(int dt, int H_I, int c_I) {
@@ -174,6 +417,50 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
                                    const int64_t* n_entries, int Q, int H_I, int c_I,
                                    float* scores, int64_t ld_scores, cudaStream_t s) {
   if (Q == 0 || ldK == 0 || nseq == 0) return cudaSuccess;
+  if (Q <= kDecMaxQ) {
+    // few queries: persistent pipelined kernel over (query, tile) units
+    CUtensorMap tmK, tmQ;
+    if (!encode_tmap_2d_bf16(&tmK, KI, (uint64_t)c_I, (uint64_t)nseq * ldK, (uint64_t)c_I * 2, 64,
+                             kTileM) ||
+        !encode_tmap_2d_bf16(&tmQ, qI, (uint64_t)c_I, (uint64_t)Q * H_I, (uint64_t)c_I * 2, 64,
+                             (uint32_t)H_I))
+      return cudaErrorInvalidValue;
+    DecParams P{};
+    P.Q = Q;
+    P.H_I = H_I;
+    P.c_I = c_I;
+    P.nseq = nseq;
+    P.ldK = ldK;
+    P.m = g.m;
+    P.vis_offset = g.vis_offset;
+    P.seq_of_q = seq_of_q;
+    P.pos = pos;
+    P.n_entries = n_entries;
+    P.w = w;
+    P.scores = scores;
+    P.ld_scores = ld_scores;
+    P.err = device_error_ptr();
+    uint32_t cols = 32;
+    while (cols < (uint32_t)(2 * H_I)) cols <<= 1;
+    P.tmem_cols = cols;
+    const int KCH = c_I / 64;
+    const size_t fixed = 1024 + 2 * (size_t)KCH * H_I * 128 + 128 * 4 + ((size_t)Q + 3) * 4 + 256;
+    const size_t per_stage = (size_t)KCH * kChunkBytesA;
+    const int stages = (int)std::min<size_t>(6, (220 * 1024 - fixed) / per_stage);
+    if (stages < 2) return cudaErrorInvalidValue;
+    P.stages = stages;
+    const size_t smem = fixed + stages * per_stage;
+    cudaError_t e = cudaFuncSetAttribute(index_decode_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int nsm = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    count_launches();
+    index_decode_kernel<<<nsm, kThreads, smem, s>>>(tmK, tmQ, P);
+    return cudaGetLastError();
+  }
   // query groups share one entry tile; many queries per call means prefill
   int G = Q >= 512 ? 256 / H_I : 1;
   if (G < 1) G = 1;

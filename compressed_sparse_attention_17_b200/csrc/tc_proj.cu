@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue ----
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // token row of the tile
-    const bool ok = tc::mbar_wait(done_bar, 0, P.err);
+    const bool ok = tc::mbar_wait_warp(done_bar, 0, P.err);
     tc::tc_fence_after();
     if (P.mode == kRaw) {
       const int64_t t = tok0 + row;

@@ -223,13 +223,13 @@ def test_index_topk_margin_rule(orc, dt, HI, cI, k):
 def test_index_topk_grouped_queries(orc, HI, cI):
     """Many queries per call: queries are processed in groups that share an
     entry tile; groups that straddle two sequences are split into passes."""
-    Q, N, k = 700, 900, 128
+    Q, N, k = 1100, 520, 128  # more queries than the persistent decode kernel takes
     rg = np.random.default_rng(12)
     qI = _spec("qIg", (Q, HI, cI), 1.0, "bf16").values()
     KI = _spec("KIg", (2, N, cI), 1.0, "bf16").values()
     w = _spec("wg", (Q, HI), 1.0, "f32").values()
     seq = np.zeros(Q, np.int32)
-    seq[400:] = rg.integers(0, 2, Q - 400)
+    seq[600:] = rg.integers(0, 2, Q - 600)
     pos = np.sort(rg.integers(0, 4 * N, Q)).astype(np.int64)
     ne = np.array([N, N - 100])
     idx, sc = _run_index(qI, w, KI, seq, pos, ne, k, "bf16", want_scores=True)
