@@ -52,21 +52,32 @@ __global__ void rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int
     inv = 1.f / sqrtf(ss / (float)c + eps);
   }
   const int64_t p = pos ? pos[row] : pos0 + row * pos_step;
+  const int npair_rot = do_rope ? r / 2 : 0;
 #pragma unroll
   for (int j = 0; j < kMaxPairsPerLane; ++j) {
     if (lane + 32 * j < c / 2) {
       int e = 2 * (lane + 32 * j);
-      float a = v[2 * j] * inv * (gain ? gain[e] : 1.f);
-      float b = v[2 * j + 1] * inv * (gain ? gain[e + 1] : 1.f);
-      if (do_rope && e >= c - r) {
-        float cs, sn;
-        rope_cs(p, (e - (c - r)) >> 1, r, base, &cs, &sn);
-        float a2 = a * cs - b * sn;
-        b = a * sn + b * cs;
-        a = a2;
+      v[2 * j] *= inv * (gain ? gain[e] : 1.f);
+      v[2 * j + 1] *= inv * (gain ? gain[e + 1] : 1.f);
+    }
+  }
+  // RoPE: lane i computes the angle of pairs i, i+32, ... once (FP64), and
+  // the owners of the rotated pairs fetch it with a shuffle
+  for (int k0 = 0; k0 < npair_rot; k0 += 32) {
+    float cs = 1.f, sn = 0.f;
+    if (k0 + lane < npair_rot) rope_cs(p, k0 + lane, r, base, &cs, &sn);
+#pragma unroll
+    for (int j = 0; j < kMaxPairsPerLane; ++j) {
+      const int e = 2 * (lane + 32 * j);
+      const int i = (e - (c - r)) >> 1;  // rotated-pair index of this lane's pair j
+      const bool mine = lane + 32 * j < c / 2 && e >= c - r && i >= k0 && i < k0 + 32;
+      const float tc_ = __shfl_sync(0xffffffffu, cs, mine ? (i - k0) : 0);
+      const float ts_ = __shfl_sync(0xffffffffu, sn, mine ? (i - k0) : 0);
+      if (mine) {
+        const float a = v[2 * j], b = v[2 * j + 1];
+        v[2 * j] = a * tc_ - b * ts_;
+        v[2 * j + 1] = a * ts_ + b * tc_;
       }
-      v[2 * j] = a;
-      v[2 * j + 1] = b;
     }
   }
   const int64_t orow = out_row ? out_row[row] : row;

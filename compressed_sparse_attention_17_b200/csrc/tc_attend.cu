@@ -133,53 +133,145 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
     }
   }
   const int64_t ldE = P.ldE;
+  const int row_bytes_e = (int)row_bytes(P.kv_dt, kDim);
+  // ---- stage the raw queries (64 KB, linear) and the index row in shared
+  //      memory with one burst of asynchronous copies ----
+  if (valid_seq && warp < 8) {
+    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(P.q + (int64_t)qi * kHeads * kDim);
+    for (int g = threadIdx.x; g < kHeads * kDim * 2 / 16; g += 256) tc::cp_async16(sQ + 16 * g, qsrc + 16 * g);
+    if (!P.dense) {
+      const int32_t* row = P.idx + (int64_t)qi * P.k;
+      if ((P.k & 3) == 0) {
+        for (int g = threadIdx.x; g < P.k / 4; g += 256) tc::cp_async16(tc::smem_u32(list + 4 * g), row + 4 * g);
+      } else {
+        for (int j = threadIdx.x; j < P.k; j += 256) list[j] = row[j];
+      }
+    }
+    tc::cp_async_wait_all();
+    tc::named_bar(2, 256);
+  }
   int64_t nsel = 0;
   if (valid_seq) {
     if (P.dense) {
       nsel = n_visible(p, P.m, P.vis_offset, min(P.n_entries[b], ldE));
-    } else {
-      // keep the slots that hold an entry inside the cache, in order
-      if (warp < 8) {
-        const int32_t* row = P.idx + (int64_t)qi * P.k;
-        __shared__ int wcount[8];
-        int base_total = 0;
-        for (int j0 = 0; j0 < P.k; j0 += 256) {
-          const int j = j0 + threadIdx.x;
-          const int32_t e = j < P.k ? row[j] : -1;
-          const bool ok = e >= 0 && e < ldE;
-          const unsigned msk = __ballot_sync(0xffffffffu, ok);
-          if (lane == 0) wcount[warp] = __popc(msk);
-          tc::named_bar(2, 256);
-          int before = 0, tot = 0;
-          for (int w = 0; w < 8; ++w) {
-            before += w < warp ? wcount[w] : 0;
-            tot += wcount[w];
-          }
-          if (ok) list[base_total + before + __popc(msk & ((1u << lane) - 1u))] = e;
-          base_total += tot;
-          tc::named_bar(2, 256);
+    } else if (warp < 8) {
+      // keep the slots that hold an entry inside the cache, in order, in
+      // place: each 256-slot chunk is read before any of it is written, and
+      // writes never pass the chunk's end
+      __shared__ int wcount[8];
+      int base_total = 0;
+      for (int j0 = 0; j0 < P.k; j0 += 256) {
+        const int j = j0 + threadIdx.x;
+        const int32_t e = j < P.k ? list[j] : -1;
+        const bool ok = e >= 0 && e < ldE;
+        const unsigned msk = __ballot_sync(0xffffffffu, ok);
+        if (lane == 0) wcount[warp] = __popc(msk);
+        tc::named_bar(2, 256);
+        int before = 0, tot = 0;
+        for (int w = 0; w < 8; ++w) {
+          before += w < warp ? wcount[w] : 0;
+          tot += wcount[w];
         }
-        if (threadIdx.x == 0) flags[2] = base_total;
+        if (ok) list[base_total + before + __popc(msk & ((1u << lane) - 1u))] = e;
+        base_total += tot;
+        tc::named_bar(2, 256);
       }
+      if (threadIdx.x == 0) flags[2] = base_total;
     }
   }
-  __syncthreads();  // RoPE table ready
-  // ---- q-hat = RoPE_p(RMSNorm(q_h) * gain) in BF16, K-major swizzled ----
-  if (valid_seq && warp < 8) {
-    for (int h = warp; h < kHeads; h += 8) {
-      const __nv_bfloat16* qr = P.q + ((int64_t)qi * kHeads + h) * kDim;
-      float v[16];
-      const uint4* src = reinterpret_cast<const uint4*>(qr + 16 * lane);
-      uint4 u0 = src[0], u1 = src[1];
-      const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&u0);
-      const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&u1);
+  if (threadIdx.x < kHeads) ref2[threadIdx.x] = P.sink[threadIdx.x] * kLog2e;
+  tc::tc_fence_before();
+  __syncthreads();  // entry list, RoPE table and TMEM address ready
+  tc::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  if (valid_seq && !P.dense) nsel = flags[2];
+
+  // ---- key slots of this CTA ----
+  const int64_t w0 = p - P.n_win + 1 > 0 ? p - P.n_win + 1 : 0;
+  const int64_t nwin = (valid_seq && P.n_win > 0) ? p - w0 + 1 : 0;
+  const int64_t nslots = valid_seq ? nsel + nwin : 0;
+  const int64_t ntiles = (nslots + kTile - 1) / kTile;
+  int64_t t_begin = 0, t_end = ntiles;
+  if (P.tiles_per_split > 0) {
+    t_begin = (int64_t)split * P.tiles_per_split;
+    t_end = min(ntiles, t_begin + P.tiles_per_split);
+  }
+
+  // gather of key tile t into sK by warps 0-7 (one 1 KB row per warp-step,
+  // 16 bytes per lane and instruction; asynchronous for BF16 rows)
+  auto issue_gather = [&](int64_t t) {
+    for (int rr = warp; rr < kTile; rr += 8) {
+      const int64_t slot = t * kTile + rr;
+      const uint8_t* row = nullptr;
+      bool mixed = false;
+      if (slot < nslots) {
+        if (slot < nsel) {
+          const int64_t e = P.dense ? slot : (int64_t)list[slot];
+          row = reinterpret_cast<const uint8_t*>(P.E) + ((int64_t)b * ldE + e) * row_bytes_e;
+          mixed = P.kv_dt == CSA_FP8_MIXED;
+        } else {
+          const int64_t j = w0 + (slot - nsel);
+          const int64_t wr = P.win_ring ? (j % P.n_win) : j;
+          if (wr < P.ldW)
+            row = reinterpret_cast<const uint8_t*>(P.win + ((int64_t)b * P.ldW + wr) * kDim);
+        }
+      }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float2 a = __bfloat1622float2(h0[i]), c2 = __bfloat1622float2(h1[i]);
-        v[2 * i] = a.x;
-        v[2 * i + 1] = a.y;
-        v[8 + 2 * i] = c2.x;
-        v[8 + 2 * i + 1] = c2.y;
+      for (int gg = 0; gg < 2; ++gg) {
+        const int g = lane + 32 * gg;  // 16-byte granule of the row: dims 8g .. 8g+7
+        const uint32_t dst = sK + (g >> 3) * 16384 + tc::sw128_offset((uint32_t)rr, (uint32_t)(g & 7));
+        if (row == nullptr) {
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+        } else if (!mixed) {
+          tc::cp_async16(dst, row + 16 * g);
+        } else {
+          uint32_t o[4];
+          if (8 * g < kMixedFp8Dims) {
+            const float sc = *reinterpret_cast<const float*>(row + kMixedScaleOffset);
+            const uint2 codes = *reinterpret_cast<const uint2*>(row + 8 * g);
+            const uint8_t* cb = reinterpret_cast<const uint8_t*>(&codes);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              __nv_bfloat162 pr = __floats2bfloat162_rn(e4m3_to_f32(cb[2 * i]) * sc,
+                                                        e4m3_to_f32(cb[2 * i + 1]) * sc);
+              o[i] = *reinterpret_cast<uint32_t*>(&pr);
+            }
+          } else {
+            const uint4 v = *reinterpret_cast<const uint4*>(row + kMixedFp8Dims + 2 * (8 * g - kMixedFp8Dims));
+            o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]),
+                       "r"(o[2]), "r"(o[3])
+                       : "memory");
+        }
+      }
+    }
+  };
+  // the first tile's rows travel while the queries are normalised
+  if (warp < 8 && t_begin < t_end) issue_gather(t_begin);
+
+  // ---- q-hat = RoPE_p(RMSNorm(q_h) * gain) in BF16, K-major swizzled, in
+  //      place: every raw value is read before any swizzled row is written ----
+  if (valid_seq && warp < 8) {
+    uint32_t raw[8][8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int h = warp + 8 * j;
+      const uint4 a = *reinterpret_cast<const uint4*>(sm + kOffQ + h * 1024 + 32 * lane);
+      const uint4 c2 = *reinterpret_cast<const uint4*>(sm + kOffQ + h * 1024 + 32 * lane + 16);
+      raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
+      raw[j][4] = c2.x; raw[j][5] = c2.y; raw[j][6] = c2.z; raw[j][7] = c2.w;
+    }
+    tc::named_bar(2, 256);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int h = warp + 8 * j;
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[j][i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
       }
       float ss = 0.f;
 #pragma unroll
@@ -216,80 +308,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       }
     }
   }
-  if (threadIdx.x < kHeads) ref2[threadIdx.x] = P.sink[threadIdx.x] * kLog2e;
-  tc::fence_proxy_async();
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
-  const uint32_t tmem = *tslot;
-  if (valid_seq && !P.dense) nsel = flags[2];
-
-  // ---- key slots of this CTA ----
-  const int64_t w0 = p - P.n_win + 1 > 0 ? p - P.n_win + 1 : 0;
-  const int64_t nwin = (valid_seq && P.n_win > 0) ? p - w0 + 1 : 0;
-  const int64_t nslots = valid_seq ? nsel + nwin : 0;
-  const int64_t ntiles = (nslots + kTile - 1) / kTile;
-  int64_t t_begin = 0, t_end = ntiles;
-  if (P.tiles_per_split > 0) {
-    t_begin = (int64_t)split * P.tiles_per_split;
-    t_end = min(ntiles, t_begin + P.tiles_per_split);
-  }
   const float scale2 = kLog2e / sqrtf((float)kDim);
   float lsum[kHeads];
 #pragma unroll
   for (int h = 0; h < kHeads; ++h) lsum[h] = 0.f;
-  const int row_bytes_e = (int)row_bytes(P.kv_dt, kDim);
 
   uint32_t phase = 0;
   for (int64_t t = t_begin; t < t_end; ++t) {
-    // ---- gather 128 key rows into sK (warps 0-3, one row per warp-step) ----
-    if (warp < 4) {
-      for (int rr = warp; rr < kTile; rr += 4) {
-        const int64_t slot = t * kTile + rr;
-        const uint8_t* row = nullptr;
-        bool mixed = false;
-        if (slot < nslots) {
-          if (slot < nsel) {
-            const int64_t e = P.dense ? slot : (int64_t)list[slot];
-            row = reinterpret_cast<const uint8_t*>(P.E) + ((int64_t)b * ldE + e) * row_bytes_e;
-            mixed = P.kv_dt == CSA_FP8_MIXED;
-          } else {
-            const int64_t j = w0 + (slot - nsel);
-            const int64_t wr = P.win_ring ? (j % P.n_win) : j;
-            if (wr < P.ldW)
-              row = reinterpret_cast<const uint8_t*>(P.win + ((int64_t)b * P.ldW + wr) * kDim);
-          }
-        }
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-          const int g = lane + 32 * gg;  // 16-byte granule of the row: dims 8g .. 8g+7
-          const uint32_t dst = sK + (g >> 3) * 16384 + tc::sw128_offset((uint32_t)rr, (uint32_t)(g & 7));
-          if (row == nullptr) {
-            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
-          } else if (!mixed) {
-            tc::cp_async16(dst, row + 16 * g);
-          } else {
-            uint32_t o[4];
-            if (8 * g < kMixedFp8Dims) {
-              const float sc = *reinterpret_cast<const float*>(row + kMixedScaleOffset);
-              const uint2 codes = *reinterpret_cast<const uint2*>(row + 8 * g);
-              const uint8_t* cb = reinterpret_cast<const uint8_t*>(&codes);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                __nv_bfloat162 pr = __floats2bfloat162_rn(e4m3_to_f32(cb[2 * i]) * sc,
-                                                          e4m3_to_f32(cb[2 * i + 1]) * sc);
-                o[i] = *reinterpret_cast<uint32_t*>(&pr);
-              }
-            } else {
-              const uint4 v = *reinterpret_cast<const uint4*>(row + kMixedFp8Dims + 2 * (8 * g - kMixedFp8Dims));
-              o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-            }
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]),
-                         "r"(o[2]), "r"(o[3])
-                         : "memory");
-          }
-        }
-      }
+    if (warp < 8) {
+      if (t > t_begin) issue_gather(t);
       tc::cp_async_wait_all();
       tc::fence_proxy_async();
     }
@@ -468,11 +495,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 
 // Merge of split partials: O = sum_s O_s 2^(m_s - m) / (2^(z'log2e - m) +
 // sum_s l_s 2^(m_s - m)), m the largest reference, fixed split order; then
-// inverse RoPE and the BF16 store. One block per (query, head).
-__global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
-  const int qi = blockIdx.x / kHeads, h = blockIdx.x % kHeads;
+// inverse RoPE and the BF16 store. One block per (query, 8 heads).
+__global__ void __launch_bounds__(256) attend_merge_kernel(Params P) {
+  __shared__ float2 rope[32];
+  const int qi = blockIdx.x >> 3, hg = blockIdx.x & 7;
   const int b = P.seq_of_q[qi];
   const int64_t p = P.pos[qi];
+  if (threadIdx.x < P.r / 2) {
+    float cs, sn;
+    rope_cs(p, threadIdx.x, P.r, P.base, &cs, &sn);
+    rope[threadIdx.x] = make_float2(cs, sn);
+  }
+  __syncthreads();
+  const bool valid_seq = b >= 0 && b < P.nseq;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = hg * 8 + warp;  // one warp per head
   const float* ml = P.part_ml + ((int64_t)qi * P.max_splits * kHeads + h) * 2;
   const float z2 = P.sink[h] * kLog2e;
   float m = z2;
@@ -480,26 +517,26 @@ __global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
   float den = exp2f(z2 - m);
   for (int sp = 0; sp < P.max_splits; ++sp)
     den += ml[(int64_t)sp * kHeads * 2 + 1] * exp2f(ml[(int64_t)sp * kHeads * 2] - m);
-  const bool valid_seq = b >= 0 && b < P.nseq;
-  for (int d0 = 2 * threadIdx.x; d0 < kDim; d0 += 256) {
+  const float inv = valid_seq ? 1.f / den : 0.f;
+  for (int d0 = 2 * lane; d0 < kDim; d0 += 64) {
     float a = 0.f, c = 0.f;
     for (int sp = 0; sp < P.max_splits; ++sp) {
       const float wgt = exp2f(ml[(int64_t)sp * kHeads * 2] - m);
-      const float* po = P.part_O + (((int64_t)qi * P.max_splits + sp) * kHeads + h) * kDim + d0;
-      a = fmaf(po[0], wgt, a);
-      c = fmaf(po[1], wgt, c);
+      const float2 po = *reinterpret_cast<const float2*>(
+          P.part_O + (((int64_t)qi * P.max_splits + sp) * kHeads + h) * kDim + d0);
+      a = fmaf(po.x, wgt, a);
+      c = fmaf(po.y, wgt, c);
     }
-    a = valid_seq ? a / den : 0.f;
-    c = valid_seq ? c / den : 0.f;
+    a *= inv;
+    c *= inv;
     if (d0 >= kDim - P.r) {
-      float cs, sn;
-      rope_cs(p, (d0 - (kDim - P.r)) >> 1, P.r, P.base, &cs, &sn);
-      const float a2 = a * cs + c * sn;
-      c = -a * sn + c * cs;
+      const float2 t = rope[(d0 - (kDim - P.r)) >> 1];
+      const float a2 = a * t.x + c * t.y;
+      c = -a * t.y + c * t.x;
       a = a2;
     }
-    __nv_bfloat162 pr = __floats2bfloat162_rn(a, c);
-    *reinterpret_cast<__nv_bfloat162*>(P.O + ((int64_t)qi * kHeads + h) * kDim + d0) = pr;
+    *reinterpret_cast<__nv_bfloat162*>(P.O + ((int64_t)qi * kHeads + h) * kDim + d0) =
+        __floats2bfloat162_rn(a, c);
   }
 }
 
@@ -577,7 +614,7 @@ cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const 
   e = cudaGetLastError();
   if (e != cudaSuccess || P.tiles_per_split == 0) return e;
   count_launches();
-  attend_merge_kernel<<<Q * kHeads, 128, 0, s>>>(P);
+  attend_merge_kernel<<<Q * 8, 256, 0, s>>>(P);
   return cudaGetLastError();
 }
 

@@ -277,7 +277,7 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap* tmW, const Params&
 }
 
 int decode_ksplit(int ntiles, int mtiles, int total_chunks, int* chunks_per_split) {
-  const int target = max(1, 148 / max(1, ntiles * mtiles));
+  const int target = min(16, max(1, 148 / max(1, ntiles * mtiles)));
   const int cps = max(1, (total_chunks + target - 1) / target);
   *chunks_per_split = cps;
   return (total_chunks + cps - 1) / cps;
