@@ -76,8 +76,9 @@ struct Params {
   __nv_bfloat16* O;
   int tiles_per_split;  // 0: one CTA per query does every tile
   int max_splits;
-  float* part_O;        // [Q][max_splits][64][512]
+  float* part_O;        // [Q][max_splits][512][64] (dim-major, as TMEM holds O^T)
   float* part_ml;       // [Q][max_splits][64][2]: reference (log2 units), sum
+  uint8_t* qhat_img;    // split mode: [Q][65536] q-hat already in the sQ layout
   int* err;
 };
 
@@ -114,14 +115,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   const bool valid_seq = b >= 0 && b < P.nseq;
   const uint32_t s_bar = tc::smem_u32(&bars[0]);
   const uint32_t o_bar = tc::smem_u32(&bars[1]);
+  const uint32_t q_bar = tc::smem_u32(&bars[2]);
+  const bool split_mode = P.tiles_per_split > 0;
 
   // ---- setup: barriers, TMEM, compacted entry list ----
   if (threadIdx.x == 0) {
     tc::mbar_init(s_bar, 1);
     tc::mbar_init(o_bar, 1);
+    tc::mbar_init(q_bar, 1);
     flags[0] = 0;
     flags[1] = 0;
     tc::fence_barrier_init();
+    if (split_mode && valid_seq) {
+      // q-hat was prepared once per query: one bulk copy of its 64 KB image
+      tc::mbar_arrive_expect_tx(q_bar, 65536u);
+      tc::bulk_copy_g2s(sQ, P.qhat_img + (int64_t)qi * 65536, 65536u, q_bar);
+    }
   }
   if (warp == 8) {
     tc::tmem_alloc(tc::smem_u32(tslot), kTmemCols);
@@ -137,8 +146,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   // ---- stage the raw queries (64 KB, linear) and the index row in shared
   //      memory with one burst of asynchronous copies ----
   if (valid_seq && warp < 8) {
-    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(P.q + (int64_t)qi * kHeads * kDim);
-    for (int g = threadIdx.x; g < kHeads * kDim * 2 / 16; g += 256) tc::cp_async16(sQ + 16 * g, qsrc + 16 * g);
+    if (!split_mode) {
+      const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(P.q + (int64_t)qi * kHeads * kDim);
+      for (int g = threadIdx.x; g < kHeads * kDim * 2 / 16; g += 256) tc::cp_async16(sQ + 16 * g, qsrc + 16 * g);
+    }
     if (!P.dense) {
       const int32_t* row = P.idx + (int64_t)qi * P.k;
       if ((P.k & 3) == 0) {
@@ -252,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 
   // ---- q-hat = RoPE_p(RMSNorm(q_h) * gain) in BF16, K-major swizzled, in
   //      place: every raw value is read before any swizzled row is written ----
-  if (valid_seq && warp < 8) {
+  if (valid_seq && warp < 8 && !split_mode) {
     uint32_t raw[8][8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -308,6 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       }
     }
   }
+  // the bulk copy of q-hat must have landed before any MMA and before exit
+  if (split_mode && valid_seq && warp == 8 && lane == 0 && !tc::mbar_wait(q_bar, 0, P.err))
+    flags[0] = 1;
   const float scale2 = kLog2e / sqrtf((float)kDim);
   float lsum[kHeads];
 #pragma unroll
@@ -437,7 +451,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       if (lane == 0) red[quad * kHeads + h] = v;
     }
     tc::named_bar(1, 128);
-    const bool split_mode = P.tiles_per_split > 0;
     if (warp == 4 || warp == 5) {
       const int h = (warp - 4) * 32 + lane;
       const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
@@ -462,12 +475,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         }
+        if (split_mode) {
+          float4* dst = reinterpret_cast<float4*>(
+              P.part_O + (((int64_t)qi * P.max_splits + split) * kDim + d) * kHeads + c0);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            dst[i / 4] = have ? make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+          continue;
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int h = c0 + i;
-          if (split_mode) {
-            P.part_O[(((int64_t)qi * P.max_splits + split) * kHeads + h) * kDim + d] = have ? o[i] : 0.f;
-          } else {
+          {
             float val = valid_seq ? o[i] * inv_den[h] : 0.f;
             if (rot) {
               // pair (d, d^1) sits in the neighbouring lane; rotate by -p
@@ -495,48 +514,127 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 
 // Merge of split partials: O = sum_s O_s 2^(m_s - m) / (2^(z'log2e - m) +
 // sum_s l_s 2^(m_s - m)), m the largest reference, fixed split order; then
-// inverse RoPE and the BF16 store. One block per (query, 8 heads).
-__global__ void __launch_bounds__(256) attend_merge_kernel(Params P) {
+// inverse RoPE and the BF16 store. One block per (query, 128 dims); thread d
+// reads its 64 heads of each split contiguously.
+__global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
   __shared__ float2 rope[32];
-  const int qi = blockIdx.x >> 3, hg = blockIdx.x & 7;
+  __shared__ float wgt[64][kHeads];  // split weights (splits <= 64)
+  __shared__ float inv[kHeads];
+  const int qi = blockIdx.x >> 2, dblk = blockIdx.x & 3;
   const int b = P.seq_of_q[qi];
   const int64_t p = P.pos[qi];
+  const bool valid_seq = b >= 0 && b < P.nseq;
+  if (threadIdx.x < P.r / 2) {
+    float cs, sn;
+    rope_cs(p, threadIdx.x, P.r, P.base, &cs, &sn);
+    rope[threadIdx.x] = make_float2(cs, sn);
+  }
+  if (threadIdx.x < kHeads) {
+    const int h = threadIdx.x;
+    const float* ml = P.part_ml + ((int64_t)qi * P.max_splits * kHeads + h) * 2;
+    const float z2 = P.sink[h] * kLog2e;
+    float m = z2;
+    for (int sp = 0; sp < P.max_splits; ++sp) m = fmaxf(m, ml[(int64_t)sp * kHeads * 2]);
+    float den = exp2f(z2 - m);
+    for (int sp = 0; sp < P.max_splits; ++sp) {
+      const float w = exp2f(ml[(int64_t)sp * kHeads * 2] - m);
+      wgt[sp][h] = w;
+      den += ml[(int64_t)sp * kHeads * 2 + 1] * w;
+    }
+    inv[h] = valid_seq ? 1.f / den : 0.f;
+  }
+  __syncthreads();
+  const int d = dblk * 128 + threadIdx.x;
+  float acc[kHeads];
+#pragma unroll
+  for (int h = 0; h < kHeads; ++h) acc[h] = 0.f;
+  for (int sp = 0; sp < P.max_splits; ++sp) {
+    const float4* src = reinterpret_cast<const float4*>(
+        P.part_O + (((int64_t)qi * P.max_splits + sp) * kDim + d) * kHeads);
+#pragma unroll
+    for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+      const float4 v = src[h4];
+      acc[4 * h4] = fmaf(v.x, wgt[sp][4 * h4], acc[4 * h4]);
+      acc[4 * h4 + 1] = fmaf(v.y, wgt[sp][4 * h4 + 1], acc[4 * h4 + 1]);
+      acc[4 * h4 + 2] = fmaf(v.z, wgt[sp][4 * h4 + 2], acc[4 * h4 + 2]);
+      acc[4 * h4 + 3] = fmaf(v.w, wgt[sp][4 * h4 + 3], acc[4 * h4 + 3]);
+    }
+  }
+  const bool rot = d >= kDim - P.r;
+  float cs = 1.f, sn = 0.f;
+  if (rot) {
+    const float2 t = rope[(d - (kDim - P.r)) >> 1];
+    cs = t.x;
+    sn = t.y;
+  }
+#pragma unroll
+  for (int h = 0; h < kHeads; ++h) {
+    float val = acc[h] * inv[h];
+    if (rot) {
+      const float other = __shfl_xor_sync(0xffffffffu, val, 1);
+      val = (d & 1) ? (-other * sn + val * cs) : (val * cs + other * sn);
+    }
+    P.O[((int64_t)qi * kHeads + h) * kDim + d] = __float2bfloat16_rn(val);
+  }
+}
+
+// q-hat = RoPE_p(RMSNorm(q_h) * gain) for every head of a query, written as
+// the exact shared-memory image the attention kernel multiplies (BF16,
+// 128-byte-swizzled K-major, 8 chunks of 64 dims x 64 heads). One block per
+// query; used when a query's keys are split over several CTAs.
+__global__ void __launch_bounds__(256) qhat_prep_kernel(Params P) {
+  __shared__ float2 rope[32];
+  const int qi = blockIdx.x;
+  const int64_t p = P.pos[qi];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < P.r / 2) {
     float cs, sn;
     rope_cs(p, threadIdx.x, P.r, P.base, &cs, &sn);
     rope[threadIdx.x] = make_float2(cs, sn);
   }
   __syncthreads();
-  const bool valid_seq = b >= 0 && b < P.nseq;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = hg * 8 + warp;  // one warp per head
-  const float* ml = P.part_ml + ((int64_t)qi * P.max_splits * kHeads + h) * 2;
-  const float z2 = P.sink[h] * kLog2e;
-  float m = z2;
-  for (int sp = 0; sp < P.max_splits; ++sp) m = fmaxf(m, ml[(int64_t)sp * kHeads * 2]);
-  float den = exp2f(z2 - m);
-  for (int sp = 0; sp < P.max_splits; ++sp)
-    den += ml[(int64_t)sp * kHeads * 2 + 1] * exp2f(ml[(int64_t)sp * kHeads * 2] - m);
-  const float inv = valid_seq ? 1.f / den : 0.f;
-  for (int d0 = 2 * lane; d0 < kDim; d0 += 64) {
-    float a = 0.f, c = 0.f;
-    for (int sp = 0; sp < P.max_splits; ++sp) {
-      const float wgt = exp2f(ml[(int64_t)sp * kHeads * 2] - m);
-      const float2 po = *reinterpret_cast<const float2*>(
-          P.part_O + (((int64_t)qi * P.max_splits + sp) * kHeads + h) * kDim + d0);
-      a = fmaf(po.x, wgt, a);
-      c = fmaf(po.y, wgt, c);
+  uint8_t* img = P.qhat_img + (int64_t)qi * 65536;
+  for (int h = warp; h < kHeads; h += 8) {
+    const __nv_bfloat16* qr = P.q + ((int64_t)qi * kHeads + h) * kDim;
+    const uint4 u0 = *reinterpret_cast<const uint4*>(qr + 16 * lane);
+    const uint4 u1 = *reinterpret_cast<const uint4*>(qr + 16 * lane + 8);
+    const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w8[i]));
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
     }
-    a *= inv;
-    c *= inv;
-    if (d0 >= kDim - P.r) {
-      const float2 t = rope[(d0 - (kDim - P.r)) >> 1];
-      const float a2 = a * t.x + c * t.y;
-      c = -a * t.y + c * t.x;
-      a = a2;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ss += v[i] * v[i];
+    ss = warp_sum(ss);
+    const float inv = 1.f / sqrtf(ss / (float)kDim + P.eps);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const int d = 16 * lane + i;
+      float a = v[i] * inv * (P.q_gain ? P.q_gain[d] : 1.f);
+      float bb = v[i + 1] * inv * (P.q_gain ? P.q_gain[d + 1] : 1.f);
+      if (d >= kDim - P.r) {
+        const float2 t = rope[(d - (kDim - P.r)) >> 1];
+        const float a2 = a * t.x - bb * t.y;
+        bb = a * t.y + bb * t.x;
+        a = a2;
+      }
+      v[i] = a;
+      v[i + 1] = bb;
     }
-    *reinterpret_cast<__nv_bfloat162*>(P.O + ((int64_t)qi * kHeads + h) * kDim + d0) =
-        __floats2bfloat162_rn(a, c);
+    const int chunk = lane >> 2;
+#pragma unroll
+    for (int gq = 0; gq < 2; ++gq) {
+      const uint32_t g = (uint32_t)((2 * lane + gq) & 7);
+      __nv_bfloat162 pk[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pk[i] = __floats2bfloat162_rn(v[8 * gq + 2 * i], v[8 * gq + 2 * i + 1]);
+      *reinterpret_cast<uint4*>(img + chunk * 8192 + tc::sw128_offset((uint32_t)h, g)) =
+          *reinterpret_cast<const uint4*>(pk);
+    }
   }
 }
 
@@ -557,7 +655,7 @@ size_t attend_tc_workspace(int Q, int64_t max_slots) {
   const int tps = choose_tiles_per_split(Q, max_slots);
   if (tps == 0) return 0;
   const int64_t splits = (max_slots + kTile - 1) / kTile;
-  return (size_t)Q * splits * kHeads * ((size_t)kDim + 2) * sizeof(float);
+  return (size_t)Q * 65536 + (size_t)Q * splits * kHeads * ((size_t)kDim + 2) * sizeof(float);
 }
 
 cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,
@@ -600,8 +698,10 @@ cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const 
     splits = (int)((max_slots + kTile - 1) / kTile);
     if (ws_bytes < attend_tc_workspace(Q, max_slots) || workspace == nullptr)
       return cudaErrorInvalidValue;
-    P.part_O = reinterpret_cast<float*>(workspace);
+    P.qhat_img = reinterpret_cast<uint8_t*>(workspace);
+    P.part_O = reinterpret_cast<float*>(P.qhat_img + (size_t)Q * 65536);
     P.part_ml = P.part_O + (size_t)Q * splits * kHeads * kDim;
+    if (splits > 64) return cudaErrorInvalidValue;
   }
   P.max_splits = splits;
   const size_t smem = (size_t)kSmemFixed + (dense ? 0 : (size_t)k * 4) + 1024;
@@ -609,12 +709,18 @@ cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const 
                                        (int)smem);
   if (e != cudaSuccess) return e;
   if (Q > 65535) return cudaErrorInvalidValue;
+  if (P.tiles_per_split > 0) {
+    count_launches();
+    qhat_prep_kernel<<<Q, 256, 0, s>>>(P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   count_launches();
   attend_tc_kernel<<<dim3((unsigned)splits, (unsigned)Q), kThreads, smem, s>>>(P);
   e = cudaGetLastError();
   if (e != cudaSuccess || P.tiles_per_split == 0) return e;
   count_launches();
-  attend_merge_kernel<<<Q * 8, 256, 0, s>>>(P);
+  attend_merge_kernel<<<Q * 4, 128, 0, s>>>(P);
   return cudaGetLastError();
 }
 
