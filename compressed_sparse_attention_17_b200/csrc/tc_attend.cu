@@ -323,9 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   if (split_mode && valid_seq && warp == 8 && lane == 0 && !tc::mbar_wait(q_bar, 0, P.err))
     flags[0] = 1;
   const float scale2 = kLog2e / sqrtf((float)kDim);
-  float lsum[kHeads];
+  // softmax/epilogue layout: warps 0-7, TMEM lane quadrant = warp % 4 (one
+  // key, or one output dim, per lane), head half = warp / 4 (32 heads)
+  const int quad = warp & 3, half = (warp >> 2) & 1;
+  const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+  float lsum[32];
 #pragma unroll
-  for (int h = 0; h < kHeads; ++h) lsum[h] = 0.f;
+  for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
 
   uint32_t phase = 0;
   for (int64_t t = t_begin; t < t_end; ++t) {
@@ -348,29 +352,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       }
       tc::mma_commit(s_bar);
     }
-    // ---- softmax on the key lanes ----
-    if (warp >= 4 && warp < 8) {
-      const int quad = warp & 3;
+    // ---- softmax on the key lanes: 32 heads per thread ----
+    if (warp < 8) {
       const int key = quad * 32 + lane;
       const int64_t slot = t * kTile + key;
       const bool kvalid = slot < nslots;
-      float s[kHeads];
+      float s[32];
       const bool ok = tc::mbar_wait_warp(s_bar, phase, P.err);
       if (!ok) flags[0] = 1;
       tc::tc_fence_after();
-      tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + kColS, s);
-      tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + kColS + 32, s + 32);
+      tc::tmem_ld32(tmem + lane_addr + kColS + half * 32, s);
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) s[h] = kvalid ? s[h] * scale2 : -INFINITY;
-      // per-head maximum over the 128 keys
+      for (int h = 0; h < 32; ++h) s[h] = kvalid ? s[h] * scale2 : -INFINITY;
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) {
+      for (int h = 0; h < 32; ++h) {
         const int mx = __reduce_max_sync(0xffffffffu, order_int(s[h]));
-        if (lane == 0) red[quad * kHeads + h] = from_order_int(mx);
+        if (lane == 0) red[quad * kHeads + half * 32 + h] = from_order_int(mx);
       }
-      tc::named_bar(1, 128);
-      if (warp == 4 || warp == 5) {
-        const int h = (warp - 4) * 32 + lane;
+      tc::named_bar(1, 256);
+      if (warp < 2) {
+        const int h = threadIdx.x;  // 0..63
         const float tmax = fmaxf(fmaxf(red[h], red[kHeads + h]), fmaxf(red[2 * kHeads + h], red[3 * kHeads + h]));
         float a = 1.f;
         if (tmax > ref2[h] + kRescaleLog2) {
@@ -380,38 +381,36 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
         }
         alpha[h] = a;
       }
-      tc::named_bar(1, 128);
-      // weights in BF16, one 128-byte row per key (heads contiguous)
+      tc::named_bar(1, 256);
+      // weights in BF16: key row of 128 bytes, this half's 4 granules
+      const float* rf = ref2 + half * 32;
+      const float* al = alpha + half * 32;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < 4; ++g) {
         uint32_t pk[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int h = 8 * g + 2 * i;
-          const float p0 = exp2f(s[h] - ref2[h]), p1 = exp2f(s[h + 1] - ref2[h + 1]);
-          lsum[h] = lsum[h] * alpha[h] + p0;
-          lsum[h + 1] = lsum[h + 1] * alpha[h + 1] + p1;
+          const float p0 = exp2f(s[h] - rf[h]), p1 = exp2f(s[h + 1] - rf[h + 1]);
+          lsum[h] = lsum[h] * al[h] + p0;
+          lsum[h + 1] = lsum[h + 1] * al[h + 1] + p1;
           __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           pk[i] = *reinterpret_cast<uint32_t*>(&pr);
         }
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sP + tc::sw128_offset((uint32_t)key, (uint32_t)g)),
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sP + tc::sw128_offset((uint32_t)key, (uint32_t)(4 * half + g))),
                      "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
                      : "memory");
       }
-      // rescale the accumulated O^T (this thread's dim lane in each block)
+      // rescale the accumulated O^T: this lane's dim in each block, this half's heads
       if (flags[1] && t > t_begin) {
-        const float* al = alpha;
 #pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < kHeads; c0 += 32) {
-            float o[32];
-            const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + kColO + blk * kHeads + c0;
-            tc::tmem_ld32(ta, o);
+          float o[32];
+          const uint32_t ta = tmem + lane_addr + kColO + blk * kHeads + half * 32;
+          tc::tmem_ld32(ta, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= al[c0 + i];
-            tc::tmem_st32(ta, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= al[i];
+          tc::tmem_st32(ta, o);
         }
       }
       tc::fence_proxy_async();
@@ -443,67 +442,69 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 
   // ---- epilogue: sums over keys, normalisation, inverse RoPE, store ----
   const bool have = t_end > t_begin && !flags[0];
-  if (warp >= 4 && warp < 8) {
-    const int quad = warp & 3;
-    // per-head sum of the weights over the 128 key lanes
-    for (int h = 0; h < kHeads; ++h) {
-      float v = warp_sum(lsum[h]);
-      if (lane == 0) red[quad * kHeads + h] = v;
+  if (warp < 8) {
+    // per-head sums over the 32 keys of this warp: butterfly transpose-
+    // reduce, lane j ends with the sum for head half*32 + j
+#pragma unroll
+    for (int off = 16, n = 16; off >= 1; off >>= 1, n >>= 1) {
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i < n) {
+          const float send = upper ? lsum[i] : lsum[i + n];
+          const float keep = upper ? lsum[i + n] : lsum[i];
+          lsum[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
     }
-    tc::named_bar(1, 128);
-    if (warp == 4 || warp == 5) {
-      const int h = (warp - 4) * 32 + lane;
+    red[quad * kHeads + half * 32 + lane] = lsum[0];
+    tc::named_bar(1, 256);
+    if (warp < 2) {
+      const int h = threadIdx.x;
       const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
-      inv_den[h] = 1.f / (l + exp2f(P.sink[h] * kLog2e - ref2[h]));
-    }
-    tc::named_bar(1, 128);
-    const int dim_in_blk = quad * 32 + lane;
-    for (int blk = 0; blk < 4; ++blk) {
-      const int d = blk * 128 + dim_in_blk;
-      float cs = 1.f, sn = 0.f;
-      const bool rot = d >= kDim - P.r;
-      if (rot) {
-        const float2 t = rope[(d - (kDim - P.r)) >> 1];
-        cs = t.x;
-        sn = t.y;
-      }
-      for (int c0 = 0; c0 < kHeads; c0 += 32) {
-        float o[32];
-        if (have) {
-          tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + kColO + blk * kHeads + c0, o);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0.f;
-        }
-        if (split_mode) {
-          float4* dst = reinterpret_cast<float4*>(
-              P.part_O + (((int64_t)qi * P.max_splits + split) * kDim + d) * kHeads + c0);
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            dst[i / 4] = have ? make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
-          continue;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int h = c0 + i;
-          {
-            float val = valid_seq ? o[i] * inv_den[h] : 0.f;
-            if (rot) {
-              // pair (d, d^1) sits in the neighbouring lane; rotate by -p
-              const float other = __shfl_xor_sync(0xffffffffu, val, 1);
-              val = (d & 1) ? (-other * sn + val * cs) : (val * cs + other * sn);
-            }
-            P.O[((int64_t)qi * kHeads + h) * kDim + d] = __float2bfloat16_rn(val);
-          }
-        }
-      }
-    }
-    if (split_mode && warp == 4) {
-      for (int h = lane; h < kHeads; h += 32) {
-        const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
+      if (split_mode) {
         float* ml = P.part_ml + (((int64_t)qi * P.max_splits + split) * kHeads + h) * 2;
         ml[0] = ref2[h];
         ml[1] = have ? l : 0.f;
+      } else {
+        inv_den[h] = 1.f / (l + exp2f(P.sink[h] * kLog2e - ref2[h]));
+      }
+    }
+    tc::named_bar(1, 256);
+    const int dim_in_blk = quad * 32 + lane;
+    for (int blk = 0; blk < 4; ++blk) {
+      const int d = blk * 128 + dim_in_blk;
+      float o[32];
+      if (have) {
+        tc::tmem_ld32(tmem + lane_addr + kColO + blk * kHeads + half * 32, o);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      }
+      if (split_mode) {
+        float4* dst = reinterpret_cast<float4*>(
+            P.part_O + (((int64_t)qi * P.max_splits + split) * kDim + d) * kHeads + half * 32);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) dst[i / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        continue;
+      }
+      float cs = 1.f, sn = 0.f;
+      const bool rot = d >= kDim - P.r;
+      if (rot) {
+        const float2 tt = rope[(d - (kDim - P.r)) >> 1];
+        cs = tt.x;
+        sn = tt.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int h = half * 32 + i;
+        float val = valid_seq ? o[i] * inv_den[h] : 0.f;
+        if (rot) {
+          // pair (d, d^1) sits in the neighbouring lane; rotate by -p
+          const float other = __shfl_xor_sync(0xffffffffu, val, 1);
+          val = (d & 1) ? (-other * sn + val * cs) : (val * cs + other * sn);
+        }
+        P.O[((int64_t)qi * kHeads + h) * kDim + d] = __float2bfloat16_rn(val);
       }
     }
   }
