@@ -296,11 +296,21 @@ def time_steps(fn, steps, warmup, device, flush, extra_events=0):
 
 
 def max_over_ranks(x: float) -> float:
+    """Largest value over all ranks (the slowest rank's time); identity
+    without a process group. NCCL groups reduce on the current GPU, others
+    (gloo) on the CPU."""
     if torch.distributed.is_initialized():
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
     return x
+
+
+def whole_job_rate(units_per_rank: int, n_ranks: int, ms_max: float) -> float:
+    """Units per second of the whole job: every rank processes its own
+    units (weak scaling), the job takes as long as its slowest rank."""
+    return n_ranks * units_per_rank / (ms_max / 1e3)
 
 
 def barrier():
@@ -426,7 +436,7 @@ def main():
     per_step_launches = launches // (args.steps + args.warmup)
     ms = statistics.mean(step_ms)
     ms_max = max_over_ranks(ms)
-    value = args.gpus * w.B / (ms_max / 1e3)
+    value = whole_job_rate(w.B, args.gpus, ms_max)
 
     # end to end through the public API from pinned host memory
     e2e_ms = None
