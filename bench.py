@@ -188,11 +188,28 @@ class Decode:
         csa.attend(inp["q"], self.sink, self.E, self.idx, self.ring, self.seq, inp["pos"],
                    self.ne, self.g, out=self.O)
 
+    def capture(self):
+        """Record one decode step (all of its library launches) as a CUDA
+        graph; replays launch the same kernels on the same buffers."""
+        self.step(self.inp)
+        torch.cuda.synchronize(self.dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step(self.inp)
+        torch.cuda.synchronize(self.dev)
+
+    def step_graph(self, ev=None):
+        self.graph.replay()
+
     def step_e2e(self):
         """Same step through the public API from pinned host buffers:
         inputs copied host->device and the output copied back."""
-        inp = {n: t.to(self.dev, non_blocking=True) for n, t in self.host.items()}
-        self.step(inp)
+        for n, t in self.host.items():
+            self.inp[n].copy_(t, non_blocking=True)
+        if getattr(self, "graph", None) is not None:
+            self.graph.replay()
+        else:
+            self.step(self.inp)
         self.host_O.copy_(self.O, non_blocking=True)
 
     @property
@@ -364,6 +381,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill secondary line")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel of a decode step from the host instead of "
+                         "replaying the step as a CUDA graph")
     ap.add_argument("--cpu-queries", type=int, default=32,
                     help="queries in the CPU-oracle sample (decode workload); 0 skips it")
     ap.add_argument("--workload", default="csa_decode_bf16",
@@ -383,7 +403,7 @@ def main():
     w = synth.WORKLOADS[args.workload]()
     if args.batch > 0:
         w = synth.WORKLOADS[args.workload](B=args.batch)
-    config = {"workload": w.name, "batch": w.B, "context": w.L, "entries_per_seq": w.n_entries,
+    config = {"workload": w.name, "launch": "host" if args.no_graph else "cuda_graph", "batch": w.B, "context": w.L, "entries_per_seq": w.n_entries,
               "m": w.m, "top_k": w.k, "window": w.n_win, "query_heads": w.H_q, "head_dim": w.c,
               "indexer_heads": w.H_I, "indexer_dim": w.c_I, "parallelism": f"dp{args.gpus}",
               "l2": "flushed (256 MiB write) before every timed step"}
@@ -428,12 +448,18 @@ def main():
     dec = Decode(w, device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     launches0 = csa.kernel_launches()
+    dec.step(dec.inp)
+    torch.cuda.synchronize(device)
+    per_step_launches = csa.kernel_launches() - launches0
+    # the indexer launch alone, for the roofline (events on the launching stream)
+    _, idx_ms = time_steps(lambda ev: dec.step(dec.inp, ev), max(5, args.steps // 2), args.warmup,
+                           device, flush, extra_events=2)
+    if not args.no_graph:
+        dec.capture()
     barrier()
     clk = Clocks(device.index).__enter__()
-    step_ms, idx_ms = time_steps(lambda ev: dec.step(dec.inp, ev), args.steps, args.warmup,
-                                 device, flush, extra_events=2)
-    launches = csa.kernel_launches() - launches0
-    per_step_launches = launches // (args.steps + args.warmup)
+    step_fn = (lambda ev: dec.step(dec.inp)) if args.no_graph else dec.step_graph
+    step_ms, _ = time_steps(step_fn, args.steps, args.warmup, device, flush)
     ms = statistics.mean(step_ms)
     ms_max = max_over_ranks(ms)
     value = whole_job_rate(w.B, args.gpus, ms_max)

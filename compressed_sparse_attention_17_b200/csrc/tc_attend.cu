@@ -108,8 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   float* inv_den = reinterpret_cast<float*>(sm + kOffInv);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qi = blockIdx.y;
-  const int split = blockIdx.x;
+  const int qi = blockIdx.x;
+  const int split = blockIdx.y;
   const int b = P.seq_of_q[qi];
   const int64_t p = P.pos[qi];
   const bool valid_seq = b >= 0 && b < P.nseq;
@@ -515,13 +515,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 
 // Merge of split partials: O = sum_s O_s 2^(m_s - m) / (2^(z'log2e - m) +
 // sum_s l_s 2^(m_s - m)), m the largest reference, fixed split order; then
-// inverse RoPE and the BF16 store. One block per (query, 128 dims); thread d
-// reads its 64 heads of each split contiguously.
-__global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
+// inverse RoPE and the BF16 store. One block per (query, 32 dims); a thread
+// reads 8 heads of one dim from each split (contiguous in the partials).
+__global__ void __launch_bounds__(256) attend_merge_kernel(Params P) {
   __shared__ float2 rope[32];
   __shared__ float wgt[64][kHeads];  // split weights (splits <= 64)
   __shared__ float inv[kHeads];
-  const int qi = blockIdx.x >> 2, dblk = blockIdx.x & 3;
+  const int qi = blockIdx.x >> 4, dblk = blockIdx.x & 15;
   const int b = P.seq_of_q[qi];
   const int64_t p = P.pos[qi];
   const bool valid_seq = b >= 0 && b < P.nseq;
@@ -530,8 +530,8 @@ __global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
     rope_cs(p, threadIdx.x, P.r, P.base, &cs, &sn);
     rope[threadIdx.x] = make_float2(cs, sn);
   }
-  if (threadIdx.x < kHeads) {
-    const int h = threadIdx.x;
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + kHeads) {
+    const int h = threadIdx.x - 64;
     const float* ml = P.part_ml + ((int64_t)qi * P.max_splits * kHeads + h) * 2;
     const float z2 = P.sink[h] * kLog2e;
     float m = z2;
@@ -545,21 +545,25 @@ __global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
     inv[h] = valid_seq ? 1.f / den : 0.f;
   }
   __syncthreads();
-  const int d = dblk * 128 + threadIdx.x;
-  float acc[kHeads];
+  // thread: dim d (lane), heads hq*8 .. hq*8+7
+  const int lane = threadIdx.x & 31, hq = threadIdx.x >> 5;
+  const int d = dblk * 32 + lane;
+  float acc[8];
 #pragma unroll
-  for (int h = 0; h < kHeads; ++h) acc[h] = 0.f;
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   for (int sp = 0; sp < P.max_splits; ++sp) {
     const float4* src = reinterpret_cast<const float4*>(
-        P.part_O + (((int64_t)qi * P.max_splits + sp) * kDim + d) * kHeads);
-#pragma unroll
-    for (int h4 = 0; h4 < kHeads / 4; ++h4) {
-      const float4 v = src[h4];
-      acc[4 * h4] = fmaf(v.x, wgt[sp][4 * h4], acc[4 * h4]);
-      acc[4 * h4 + 1] = fmaf(v.y, wgt[sp][4 * h4 + 1], acc[4 * h4 + 1]);
-      acc[4 * h4 + 2] = fmaf(v.z, wgt[sp][4 * h4 + 2], acc[4 * h4 + 2]);
-      acc[4 * h4 + 3] = fmaf(v.w, wgt[sp][4 * h4 + 3], acc[4 * h4 + 3]);
-    }
+        P.part_O + (((int64_t)qi * P.max_splits + sp) * kDim + d) * kHeads + hq * 8);
+    const float4 v0 = src[0], v1 = src[1];
+    const float* wv = &wgt[sp][hq * 8];
+    acc[0] = fmaf(v0.x, wv[0], acc[0]);
+    acc[1] = fmaf(v0.y, wv[1], acc[1]);
+    acc[2] = fmaf(v0.z, wv[2], acc[2]);
+    acc[3] = fmaf(v0.w, wv[3], acc[3]);
+    acc[4] = fmaf(v1.x, wv[4], acc[4]);
+    acc[5] = fmaf(v1.y, wv[5], acc[5]);
+    acc[6] = fmaf(v1.z, wv[6], acc[6]);
+    acc[7] = fmaf(v1.w, wv[7], acc[7]);
   }
   const bool rot = d >= kDim - P.r;
   float cs = 1.f, sn = 0.f;
@@ -569,8 +573,9 @@ __global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
     sn = t.y;
   }
 #pragma unroll
-  for (int h = 0; h < kHeads; ++h) {
-    float val = acc[h] * inv[h];
+  for (int i = 0; i < 8; ++i) {
+    const int h = hq * 8 + i;
+    float val = acc[i] * inv[h];
     if (rot) {
       const float other = __shfl_xor_sync(0xffffffffu, val, 1);
       val = (d & 1) ? (-other * sn + val * cs) : (val * cs + other * sn);
@@ -582,10 +587,11 @@ __global__ void __launch_bounds__(128) attend_merge_kernel(Params P) {
 // q-hat = RoPE_p(RMSNorm(q_h) * gain) for every head of a query, written as
 // the exact shared-memory image the attention kernel multiplies (BF16,
 // 128-byte-swizzled K-major, 8 chunks of 64 dims x 64 heads). One block per
-// query; used when a query's keys are split over several CTAs.
+// (query, 8 heads), one warp per head; used when a query's keys are split
+// over several CTAs.
 __global__ void __launch_bounds__(256) qhat_prep_kernel(Params P) {
   __shared__ float2 rope[32];
-  const int qi = blockIdx.x;
+  const int qi = blockIdx.x >> 3, hg = blockIdx.x & 7;
   const int64_t p = P.pos[qi];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < P.r / 2) {
@@ -595,7 +601,8 @@ __global__ void __launch_bounds__(256) qhat_prep_kernel(Params P) {
   }
   __syncthreads();
   uint8_t* img = P.qhat_img + (int64_t)qi * 65536;
-  for (int h = warp; h < kHeads; h += 8) {
+  {
+    const int h = hg * 8 + warp;
     const __nv_bfloat16* qr = P.q + ((int64_t)qi * kHeads + h) * kDim;
     const uint4 u0 = *reinterpret_cast<const uint4*>(qr + 16 * lane);
     const uint4 u1 = *reinterpret_cast<const uint4*>(qr + 16 * lane + 8);
@@ -709,19 +716,18 @@ cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const 
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  if (Q > 65535) return cudaErrorInvalidValue;
   if (P.tiles_per_split > 0) {
     count_launches();
-    qhat_prep_kernel<<<Q, 256, 0, s>>>(P);
+    qhat_prep_kernel<<<Q * 8, 256, 0, s>>>(P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   count_launches();
-  attend_tc_kernel<<<dim3((unsigned)splits, (unsigned)Q), kThreads, smem, s>>>(P);
+  attend_tc_kernel<<<dim3((unsigned)Q, (unsigned)splits), kThreads, smem, s>>>(P);
   e = cudaGetLastError();
   if (e != cudaSuccess || P.tiles_per_split == 0) return e;
   count_launches();
-  attend_merge_kernel<<<Q * 4, 128, 0, s>>>(P);
+  attend_merge_kernel<<<Q * 16, 256, 0, s>>>(P);
   return cudaGetLastError();
 }
 

@@ -225,6 +225,9 @@ struct UnitWalk {
   }
 };
 
+// HREG = H_I when the head weights of the current query are kept in
+// registers (reloaded when the query changes), 0 for read-through loads.
+template <int HREG>
 __global__ void __launch_bounds__(kThreads, 1)
     index_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                         DecParams P) {
@@ -374,23 +377,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t nv = 0;
     float* out = nullptr;
     const float* wq = nullptr;
+    float wr[HREG > 0 ? HREG : 1];
     for (int i = 0; i < nunits; ++i, wk.next()) {
       const int q = wk.q;
       if (q != last_q) {
         nv = dec_nvis(P, q);
         out = P.scores + (int64_t)q * P.ld_scores;
         wq = P.w + (int64_t)q * P.H_I;
+        if (HREG > 0) {
+#pragma unroll
+          for (int h = 0; h < HREG; h += 4) {
+            const float4 t4 = __ldg(reinterpret_cast<const float4*>(wq + h));
+            wr[h] = t4.x;
+            wr[h + 1] = t4.y;
+            wr[h + 2] = t4.z;
+            wr[h + 3] = t4.w;
+          }
+        }
         last_q = q;
       }
       const int a = i & 1;
       if (!tc::mbar_wait_warp(accfull(a), (i >> 1) & 1, P.err)) break;
       tc::tc_fence_after();
       float acc = 0.f;
-      for (int h0 = 0; h0 < P.H_I; h0 += 16) {
-        float v[16];
-        tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * P.H_I + h0), v);
+      if (HREG > 0) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc = fmaf(__ldg(wq + h0 + j), fmaxf(v[j], 0.f), acc);
+        for (int h0 = 0; h0 < (HREG > 0 ? HREG : 16); h0 += 32) {
+          float v[32];
+          tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * HREG + h0), v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc = fmaf(wr[h0 + j], fmaxf(v[j], 0.f), acc);
+        }
+      } else {
+        for (int h0 = 0; h0 < P.H_I; h0 += 16) {
+          float v[16];
+          tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * P.H_I + h0), v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc = fmaf(__ldg(wq + h0 + j), fmaxf(v[j], 0.f), acc);
+        }
       }
       tc::tc_fence_before();
       __syncwarp();
@@ -450,15 +474,17 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
     if (stages < 2) return cudaErrorInvalidValue;
     P.stages = stages;
     const size_t smem = fixed + stages * per_stage;
-    cudaError_t e = cudaFuncSetAttribute(index_decode_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // w rows are read as float4 in the register path: 16-byte aligned rows
+    const bool wreg = H_I == 64 && (reinterpret_cast<uintptr_t>(w) & 15) == 0;
+    auto kern = wreg ? index_decode_kernel<64> : index_decode_kernel<0>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int nsm = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     count_launches();
-    index_decode_kernel<<<nsm, kThreads, smem, s>>>(tmK, tmQ, P);
+    kern<<<nsm, kThreads, smem, s>>>(tmK, tmQ, P);
     return cudaGetLastError();
   }
   // query groups share one entry tile; many queries per call means prefill

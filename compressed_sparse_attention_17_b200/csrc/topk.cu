@@ -54,7 +54,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) 
 }
 
 struct SelectScratch {
-  int hist_w[kWarps][256];
+  int hist[256];
   int scan[kWarps];
   uint32_t prefix;
   int remaining;
@@ -68,11 +68,19 @@ __device__ void radix_threshold(const uint32_t* keys, int n, int k, SelectScratc
   uint32_t prefix = 0, mask = 0;
   int remaining = k;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < kWarps * 256; i += kThreads) (&S.hist_w[0][0])[i] = 0;
+    if (tid < 256) S.hist[tid] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kThreads) {
-      const uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&S.hist_w[wid][(key >> shift) & 255u], 1);
+    // warp-aggregated increments: lanes with the same digit add once
+    for (int i0 = wid * 32; i0 < n; i0 += kThreads) {
+      const int i = i0 + lane;
+      const uint32_t key = i < n ? keys[i] : 0u;
+      const bool act = i < n && (key & mask) == prefix;
+      const unsigned am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t dg = (key >> shift) & 255u;
+        const unsigned peers = __match_any_sync(am, dg);
+        if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&S.hist[dg], __popc(peers));
+      }
     }
     __syncthreads();
     if (wid == 0) {
@@ -80,9 +88,7 @@ __device__ void radix_threshold(const uint32_t* keys, int n, int k, SelectScratc
       int cnt[8], sum = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int dg = 255 - (8 * lane + j);
-        int c = 0;
-        for (int w = 0; w < kWarps; ++w) c += S.hist_w[w][dg];
+        const int c = S.hist[255 - (8 * lane + j)];
         cnt[j] = c;
         sum += c;
       }
