@@ -253,6 +253,25 @@ def test_index_topk_many_entries_bit_exact(orc, k):
     np.testing.assert_array_equal(idx, want)
 
 
+@pytest.mark.parametrize("N,k", [(1500, 700), (40000, 1024), (70000, 512)])
+def test_index_topk_equal_scores(orc, N, k):
+    """Zero indexer queries make every score 0: all visible entries tie and
+    the lowest k_eff indices are kept. One bin then holds every key, so the
+    exact ranking of that bin (1,500 entries), the radix selection over a
+    whole multi-CTA row (40,000) and chunked rows (70,000) all run."""
+    qI, w, KI, seq, pos, ne = _index_inputs(6, 4, 32, 2, N, "f32", integer=True, seed=11)
+    qI[:] = 0.0
+    pos[:] = [4 * N + 3, 4 * k - 1, 4 * k + 3, 4 * (N // 2), 7, 4 * N - 9]
+    idx = _run_index(qI, w, KI, seq, pos, ne, k, "f32").cpu().numpy()
+    want = orc.index_topk(qI, w, KI, seq, pos, ne, m=4, k=k)["idx"]
+    np.testing.assert_array_equal(idx, want)
+    for q in range(len(pos)):
+        nv = orc.visible_entries(pos[q], 4, 1, ne[seq[q]])
+        ke = min(k, nv)
+        np.testing.assert_array_equal(idx[q, :ke], np.arange(ke))
+        assert (idx[q, ke:] == -1).all()
+
+
 def test_index_topk_no_visible_entries(orc):
     qI, w, KI, seq, pos, ne = _index_inputs(8, 4, 32, 1, 50, "f32", seed=5)
     pos[:] = [0, 1, 2, 3, 4, 5, 6, 7]
