@@ -496,7 +496,7 @@ def main():
             traffic = None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic,
-                "kernel": "csa_index_topk (decode, all 32 queries)",
+                "kernel": f"csa_index_topk (decode, all {w.B} queries)",
                 "kernel_ms": idx_avg, "algorithmic_bytes": idx_bytes,
                 "peak_source": f"{peak_kind} HBM copy bandwidth"}
 

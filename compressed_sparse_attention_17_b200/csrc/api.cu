@@ -227,8 +227,8 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
 }
 
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win) {
-  if (Q <= 0 || k < 0 || n_win < 0 || c != 512 || H_q != 64) return 0;
-  return csa::attend_tc_workspace(Q, (int64_t)k + n_win);
+  (void)Q, (void)H_q, (void)c, (void)k, (void)n_win;
+  return 0;
 }
 
 static csa_status attend_common(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype,
@@ -251,15 +251,20 @@ static csa_status attend_common(const csa_geom* g, csa_dtype q_dtype, csa_dtype 
   for (const void* p : ptrs)
     if (!aligned16(p)) return CSA_ERR_INVALID_ARG;
   if (!aligned16(workspace)) return CSA_ERR_INVALID_ARG;
-  if (csa::attend_tc_supported(q_dtype, kv_dtype, g->c, H_q, dense ? 0 : k, g->rope_dims)) {
-    const int64_t max_slots = (dense ? ldE : (int64_t)k) + g->n_win;
-    const size_t need = csa::attend_tc_workspace(Q, max_slots);
-    if (need > 0 && (!workspace || ws_bytes < need)) return CSA_ERR_INVALID_ARG;
+  (void)workspace, (void)ws_bytes;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int kk = dense ? 0 : k;
+  // small batches: one cluster per query (batch-invariant); large batches:
+  // one CTA per query
+  const bool tc_big = csa::attend_tc_supported(q_dtype, kv_dtype, g->c, H_q, kk, g->rope_dims);
+  if (csa::attend_cluster_supported(q_dtype, kv_dtype, g->c, H_q, kk, g->rope_dims) &&
+      (Q < CSA_ATTEND_INVARIANT_Q || !tc_big))
+    return cuda_status(csa::launch_attend_cluster(*g, kv_dtype, q, q_gain, sink, E, ldE, nseq,
+                                                  n_entries, idx, kk, dense, win, ldW, seq_of_q,
+                                                  pos, Q, O, s));
+  if (tc_big)
     return cuda_status(csa::launch_attend_tc(*g, kv_dtype, q, q_gain, sink, E, ldE, nseq, n_entries,
-                                             idx, dense ? 0 : k, dense, win, ldW, seq_of_q, pos, Q,
-                                             O, workspace, ws_bytes,
-                                             reinterpret_cast<cudaStream_t>(stream)));
-  }
+                                             idx, kk, dense, win, ldW, seq_of_q, pos, Q, O, s));
   if (!csa::attend_simt_supported(g->c, H_q)) return CSA_ERR_UNSUPPORTED;
   return cuda_status(launch_attend_simt(*g, q_dtype, kv_dtype, q, q_gain, sink, E, ldE, nseq,
                                         n_entries, idx, k, dense, win, ldW, seq_of_q, pos, Q, H_q, O,
@@ -277,8 +282,8 @@ csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, 
 }
 
 size_t hca_attend_workspace_size(int Q, int H_q, int c, int64_t ldE, int n_win) {
-  if (Q <= 0 || ldE < 0 || n_win < 0 || c != 512 || H_q != 64) return 0;
-  return csa::attend_tc_workspace(Q, ldE + n_win);
+  (void)Q, (void)H_q, (void)c, (void)ldE, (void)n_win;
+  return 0;
 }
 
 csa_status hca_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,

@@ -31,6 +31,18 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
+// BF16 pairs packed in 32-bit words (low half = first element), handled in
+// registers: taking the address of a local array to reinterpret it would put
+// the array in local memory.
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+__device__ __forceinline__ uint8_t byte_of(uint32_t u, int i) { return (uint8_t)(u >> (8 * i)); }
+
 // E4M3 code -> float (exact).
 __device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
   __nv_fp8_e4m3 v;

@@ -66,14 +66,20 @@ cudaError_t launch_compress_tc(const csa_geom& g, const void* H, int64_t T, int 
 cudaError_t launch_decode_proj_tc(const csa_geom& g, const void* h, const int64_t* pos, int B,
                                   int d, const void* const* W, float* part, float* state,
                                   cudaStream_t s);
+// Shared-KV attention, one thread-block cluster per query (tc_attend_cluster.cu).
+int attend_cluster_size(int64_t max_slots);
+bool attend_cluster_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_dims);
+cudaError_t launch_attend_cluster(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,
+                                  const float* sink, const void* E, int64_t ldE, int nseq,
+                                  const int64_t* n_entries, const int32_t* idx, int k, int dense,
+                                  const void* win, int64_t ldW, const int32_t* seq_of_q,
+                                  const int64_t* pos, int Q, void* O, cudaStream_t s);
 bool attend_tc_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_dims);
-size_t attend_tc_workspace(int Q, int64_t max_slots);
 cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,
                              const float* sink, const void* E, int64_t ldE, int nseq,
                              const int64_t* n_entries, const int32_t* idx, int k, int dense,
                              const void* win, int64_t ldW, const int32_t* seq_of_q,
-                             const int64_t* pos, int Q, void* O, void* workspace,
-                             size_t ws_bytes, cudaStream_t s);
+                             const int64_t* pos, int Q, void* O, cudaStream_t s);
 // dense != 0: HCA (all visible entries); else CSA with idx [Q, k].
 cudaError_t launch_attend_simt(const csa_geom& g, int q_dt, int kv_dt, const void* q,
                                const float* q_gain, const float* sink, const void* E,

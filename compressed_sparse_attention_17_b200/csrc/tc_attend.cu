@@ -20,9 +20,9 @@
 // 2^8, so the FP32 sums and the BF16 weights neither overflow nor lose
 // range, and the result is the exact softmax up to rounding.
 //
-// Small batches split each query's key list across CTAs (fixed split
-// boundaries) and merge the partial (m, l, O) in a fixed order, so a
-// query's result does not depend on the batch it is in.
+// This kernel serves large batches (prefill), one CTA per query; small
+// batches run on the cluster kernel (tc_attend_cluster.cu), which splits a
+// query's keys over several CTAs.
 //
 // Warps (288 threads): 0-3 gather key rows (cp.async) and prepare Qhat with
 // 4-7; 4-7 run the softmax and the output epilogue (TMEM lane quadrant =
@@ -74,11 +74,6 @@ struct Params {
   const int32_t* seq_of_q;
   const int64_t* pos;
   __nv_bfloat16* O;
-  int tiles_per_split;  // 0: one CTA per query does every tile
-  int max_splits;
-  float* part_O;        // [Q][max_splits][512][64] (dim-major, as TMEM holds O^T)
-  float* part_ml;       // [Q][max_splits][64][2]: reference (log2 units), sum
-  uint8_t* qhat_img;    // split mode: [Q][65536] q-hat already in the sQ layout
   int* err;
 };
 
@@ -109,28 +104,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qi = blockIdx.x;
-  const int split = blockIdx.y;
   const int b = P.seq_of_q[qi];
   const int64_t p = P.pos[qi];
   const bool valid_seq = b >= 0 && b < P.nseq;
   const uint32_t s_bar = tc::smem_u32(&bars[0]);
   const uint32_t o_bar = tc::smem_u32(&bars[1]);
-  const uint32_t q_bar = tc::smem_u32(&bars[2]);
-  const bool split_mode = P.tiles_per_split > 0;
 
   // ---- setup: barriers, TMEM, compacted entry list ----
   if (threadIdx.x == 0) {
     tc::mbar_init(s_bar, 1);
     tc::mbar_init(o_bar, 1);
-    tc::mbar_init(q_bar, 1);
     flags[0] = 0;
     flags[1] = 0;
     tc::fence_barrier_init();
-    if (split_mode && valid_seq) {
-      // q-hat was prepared once per query: one bulk copy of its 64 KB image
-      tc::mbar_arrive_expect_tx(q_bar, 65536u);
-      tc::bulk_copy_g2s(sQ, P.qhat_img + (int64_t)qi * 65536, 65536u, q_bar);
-    }
   }
   if (warp == 8) {
     tc::tmem_alloc(tc::smem_u32(tslot), kTmemCols);
@@ -146,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   // ---- stage the raw queries (64 KB, linear) and the index row in shared
   //      memory with one burst of asynchronous copies ----
   if (valid_seq && warp < 8) {
-    if (!split_mode) {
+    {
       const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(P.q + (int64_t)qi * kHeads * kDim);
       for (int g = threadIdx.x; g < kHeads * kDim * 2 / 16; g += 256) tc::cp_async16(sQ + 16 * g, qsrc + 16 * g);
     }
@@ -202,11 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   const int64_t nwin = (valid_seq && P.n_win > 0) ? p - w0 + 1 : 0;
   const int64_t nslots = valid_seq ? nsel + nwin : 0;
   const int64_t ntiles = (nslots + kTile - 1) / kTile;
-  int64_t t_begin = 0, t_end = ntiles;
-  if (P.tiles_per_split > 0) {
-    t_begin = (int64_t)split * P.tiles_per_split;
-    t_end = min(ntiles, t_begin + P.tiles_per_split);
-  }
+  const int64_t t_begin = 0, t_end = ntiles;
 
   // gather of key tile t into sK by warps 0-7 (one 1 KB row per warp-step,
   // 16 bytes per lane and instruction; asynchronous for BF16 rows)
@@ -263,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
 
   // ---- q-hat = RoPE_p(RMSNorm(q_h) * gain) in BF16, K-major swizzled, in
   //      place: every raw value is read before any swizzled row is written ----
-  if (valid_seq && warp < 8 && !split_mode) {
+  if (valid_seq && warp < 8) {
     uint32_t raw[8][8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -320,8 +302,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
     }
   }
   // the bulk copy of q-hat must have landed before any MMA and before exit
-  if (split_mode && valid_seq && warp == 8 && lane == 0 && !tc::mbar_wait(q_bar, 0, P.err))
-    flags[0] = 1;
   const float scale2 = kLog2e / sqrtf((float)kDim);
   // softmax/epilogue layout: warps 0-7, TMEM lane quadrant = warp % 4 (one
   // key, or one output dim, per lane), head half = warp / 4 (32 heads)
@@ -462,13 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
     if (warp < 2) {
       const int h = threadIdx.x;
       const float l = red[h] + red[kHeads + h] + red[2 * kHeads + h] + red[3 * kHeads + h];
-      if (split_mode) {
-        float* ml = P.part_ml + (((int64_t)qi * P.max_splits + split) * kHeads + h) * 2;
-        ml[0] = ref2[h];
-        ml[1] = have ? l : 0.f;
-      } else {
-        inv_den[h] = 1.f / (l + exp2f(P.sink[h] * kLog2e - ref2[h]));
-      }
+      inv_den[h] = 1.f / (l + exp2f(P.sink[h] * kLog2e - ref2[h]));
     }
     tc::named_bar(1, 256);
     const int dim_in_blk = quad * 32 + lane;
@@ -480,13 +454,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
-      }
-      if (split_mode) {
-        float4* dst = reinterpret_cast<float4*>(
-            P.part_O + (((int64_t)qi * P.max_splits + split) * kDim + d) * kHeads + half * 32);
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) dst[i / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-        continue;
       }
       float cs = 1.f, sn = 0.f;
       const bool rot = d >= kDim - P.r;
@@ -513,145 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   if (warp == 8) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Merge of split partials: O = sum_s O_s 2^(m_s - m) / (2^(z'log2e - m) +
-// sum_s l_s 2^(m_s - m)), m the largest reference, fixed split order; then
-// inverse RoPE and the BF16 store. One block per (query, 32 dims); a thread
-// reads 8 heads of one dim from each split (contiguous in the partials).
-__global__ void __launch_bounds__(256) attend_merge_kernel(Params P) {
-  __shared__ float2 rope[32];
-  __shared__ float wgt[64][kHeads];  // split weights (splits <= 64)
-  __shared__ float inv[kHeads];
-  const int qi = blockIdx.x >> 4, dblk = blockIdx.x & 15;
-  const int b = P.seq_of_q[qi];
-  const int64_t p = P.pos[qi];
-  const bool valid_seq = b >= 0 && b < P.nseq;
-  if (threadIdx.x < P.r / 2) {
-    float cs, sn;
-    rope_cs(p, threadIdx.x, P.r, P.base, &cs, &sn);
-    rope[threadIdx.x] = make_float2(cs, sn);
-  }
-  if (threadIdx.x >= 64 && threadIdx.x < 64 + kHeads) {
-    const int h = threadIdx.x - 64;
-    const float* ml = P.part_ml + ((int64_t)qi * P.max_splits * kHeads + h) * 2;
-    const float z2 = P.sink[h] * kLog2e;
-    float m = z2;
-    for (int sp = 0; sp < P.max_splits; ++sp) m = fmaxf(m, ml[(int64_t)sp * kHeads * 2]);
-    float den = exp2f(z2 - m);
-    for (int sp = 0; sp < P.max_splits; ++sp) {
-      const float w = exp2f(ml[(int64_t)sp * kHeads * 2] - m);
-      wgt[sp][h] = w;
-      den += ml[(int64_t)sp * kHeads * 2 + 1] * w;
-    }
-    inv[h] = valid_seq ? 1.f / den : 0.f;
-  }
-  __syncthreads();
-  // thread: dim d (lane), heads hq*8 .. hq*8+7
-  const int lane = threadIdx.x & 31, hq = threadIdx.x >> 5;
-  const int d = dblk * 32 + lane;
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int sp = 0; sp < P.max_splits; ++sp) {
-    const float4* src = reinterpret_cast<const float4*>(
-        P.part_O + (((int64_t)qi * P.max_splits + sp) * kDim + d) * kHeads + hq * 8);
-    const float4 v0 = src[0], v1 = src[1];
-    const float* wv = &wgt[sp][hq * 8];
-    acc[0] = fmaf(v0.x, wv[0], acc[0]);
-    acc[1] = fmaf(v0.y, wv[1], acc[1]);
-    acc[2] = fmaf(v0.z, wv[2], acc[2]);
-    acc[3] = fmaf(v0.w, wv[3], acc[3]);
-    acc[4] = fmaf(v1.x, wv[4], acc[4]);
-    acc[5] = fmaf(v1.y, wv[5], acc[5]);
-    acc[6] = fmaf(v1.z, wv[6], acc[6]);
-    acc[7] = fmaf(v1.w, wv[7], acc[7]);
-  }
-  const bool rot = d >= kDim - P.r;
-  float cs = 1.f, sn = 0.f;
-  if (rot) {
-    const float2 t = rope[(d - (kDim - P.r)) >> 1];
-    cs = t.x;
-    sn = t.y;
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int h = hq * 8 + i;
-    float val = acc[i] * inv[h];
-    if (rot) {
-      const float other = __shfl_xor_sync(0xffffffffu, val, 1);
-      val = (d & 1) ? (-other * sn + val * cs) : (val * cs + other * sn);
-    }
-    P.O[((int64_t)qi * kHeads + h) * kDim + d] = __float2bfloat16_rn(val);
-  }
-}
-
-// q-hat = RoPE_p(RMSNorm(q_h) * gain) for every head of a query, written as
-// the exact shared-memory image the attention kernel multiplies (BF16,
-// 128-byte-swizzled K-major, 8 chunks of 64 dims x 64 heads). One block per
-// (query, 8 heads), one warp per head; used when a query's keys are split
-// over several CTAs.
-__global__ void __launch_bounds__(256) qhat_prep_kernel(Params P) {
-  __shared__ float2 rope[32];
-  const int qi = blockIdx.x >> 3, hg = blockIdx.x & 7;
-  const int64_t p = P.pos[qi];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x < P.r / 2) {
-    float cs, sn;
-    rope_cs(p, threadIdx.x, P.r, P.base, &cs, &sn);
-    rope[threadIdx.x] = make_float2(cs, sn);
-  }
-  __syncthreads();
-  uint8_t* img = P.qhat_img + (int64_t)qi * 65536;
-  {
-    const int h = hg * 8 + warp;
-    const __nv_bfloat16* qr = P.q + ((int64_t)qi * kHeads + h) * kDim;
-    const uint4 u0 = *reinterpret_cast<const uint4*>(qr + 16 * lane);
-    const uint4 u1 = *reinterpret_cast<const uint4*>(qr + 16 * lane + 8);
-    const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w8[i]));
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
-    }
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) ss += v[i] * v[i];
-    ss = warp_sum(ss);
-    const float inv = 1.f / sqrtf(ss / (float)kDim + P.eps);
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const int d = 16 * lane + i;
-      float a = v[i] * inv * (P.q_gain ? P.q_gain[d] : 1.f);
-      float bb = v[i + 1] * inv * (P.q_gain ? P.q_gain[d + 1] : 1.f);
-      if (d >= kDim - P.r) {
-        const float2 t = rope[(d - (kDim - P.r)) >> 1];
-        const float a2 = a * t.x - bb * t.y;
-        bb = a * t.y + bb * t.x;
-        a = a2;
-      }
-      v[i] = a;
-      v[i + 1] = bb;
-    }
-    const int chunk = lane >> 2;
-#pragma unroll
-    for (int gq = 0; gq < 2; ++gq) {
-      const uint32_t g = (uint32_t)((2 * lane + gq) & 7);
-      __nv_bfloat162 pk[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) pk[i] = __floats2bfloat162_rn(v[8 * gq + 2 * i], v[8 * gq + 2 * i + 1]);
-      *reinterpret_cast<uint4*>(img + chunk * 8192 + tc::sw128_offset((uint32_t)h, g)) =
-          *reinterpret_cast<const uint4*>(pk);
-    }
-  }
-}
-
-int choose_tiles_per_split(int Q, int64_t max_slots) {
-  const int64_t tiles = (max_slots + kTile - 1) / kTile;
-  // few queries: one tile per CTA so that every SM has work
-  return ((int64_t)Q * tiles <= 4 * 148) ? 1 : 0;
-}
-
 }  // namespace
 
 bool attend_tc_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_dims) {
@@ -659,21 +487,12 @@ bool attend_tc_supported(int q_dt, int kv_dt, int c, int H_q, int k, int rope_di
          H_q == kHeads && k <= CSA_MAX_TOPK && rope_dims % 32 == 0 && rope_dims <= 64;
 }
 
-size_t attend_tc_workspace(int Q, int64_t max_slots) {
-  const int tps = choose_tiles_per_split(Q, max_slots);
-  if (tps == 0) return 0;
-  const int64_t splits = (max_slots + kTile - 1) / kTile;
-  return (size_t)Q * 65536 + (size_t)Q * splits * kHeads * ((size_t)kDim + 2) * sizeof(float);
-}
-
 cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const float* q_gain,
                              const float* sink, const void* E, int64_t ldE, int nseq,
                              const int64_t* n_entries, const int32_t* idx, int k, int dense,
                              const void* win, int64_t ldW, const int32_t* seq_of_q,
-                             const int64_t* pos, int Q, void* O, void* workspace,
-                             size_t ws_bytes, cudaStream_t s) {
+                             const int64_t* pos, int Q, void* O, cudaStream_t s) {
   if (Q == 0) return cudaSuccess;
-  const int64_t max_slots = (dense ? ldE : (int64_t)k) + g.n_win;
   Params P{};
   P.Q = Q;
   P.r = g.rope_dims;
@@ -700,34 +519,12 @@ cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const 
   P.pos = pos;
   P.O = reinterpret_cast<__nv_bfloat16*>(O);
   P.err = device_error_ptr();
-  P.tiles_per_split = choose_tiles_per_split(Q, max_slots);
-  int splits = 1;
-  if (P.tiles_per_split > 0) {
-    splits = (int)((max_slots + kTile - 1) / kTile);
-    if (ws_bytes < attend_tc_workspace(Q, max_slots) || workspace == nullptr)
-      return cudaErrorInvalidValue;
-    P.qhat_img = reinterpret_cast<uint8_t*>(workspace);
-    P.part_O = reinterpret_cast<float*>(P.qhat_img + (size_t)Q * 65536);
-    P.part_ml = P.part_O + (size_t)Q * splits * kHeads * kDim;
-    if (splits > 64) return cudaErrorInvalidValue;
-  }
-  P.max_splits = splits;
   const size_t smem = (size_t)kSmemFixed + (dense ? 0 : (size_t)k * 4) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  if (P.tiles_per_split > 0) {
-    count_launches();
-    qhat_prep_kernel<<<Q * 8, 256, 0, s>>>(P);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   count_launches();
-  attend_tc_kernel<<<dim3((unsigned)Q, (unsigned)splits), kThreads, smem, s>>>(P);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || P.tiles_per_split == 0) return e;
-  count_launches();
-  attend_merge_kernel<<<Q * 16, 256, 0, s>>>(P);
+  attend_tc_kernel<<<(unsigned)Q, kThreads, smem, s>>>(P);
   return cudaGetLastError();
 }
 

@@ -277,10 +277,16 @@ csa_status csa_index_topk_noalloc(const csa_geom* g, csa_dtype dtype, const void
  *   win   [nseq, ldW, c] kv_dtype (F32 or BF16), rows already prepared
  *         (csa_rmsnorm_rope); row of position j = j (win_ring = 0, ldW > p)
  *         or j mod n_win (win_ring = 1, ldW >= n_win).
- * workspace: csa_attend_workspace_size() bytes (non-zero when few queries
- * are spread over more CTAs than one per query: the per-split partial
- * results live there).
+ * workspace: csa_attend_workspace_size() bytes, currently 0 for every
+ * shape (the kernels keep their partial results on chip); callers may pass
+ * NULL with ws_bytes = 0.
+ * Results for a query do not depend on the other queries of the call while
+ * Q < CSA_ATTEND_INVARIANT_Q (one thread-block cluster per query, split
+ * boundaries fixed by k and n_win alone); larger calls run one CTA per
+ * query, whose accumulation order differs (results agree within the
+ * attention tolerance, not bit for bit).
  * --------------------------------------------------------------------- */
+#define CSA_ATTEND_INVARIANT_Q 1024
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win);
 csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,
                       const float* q_gain, const float* sink, const void* E, int64_t ldE,
@@ -293,7 +299,7 @@ csa_status csa_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, 
  * causally available entry is read, no indexer). Same as csa_attend with
  * J = { E[b, s] : s < n_vis(q) } U window, n_vis computed from g->m and
  * g->vis_offset and clipped to n_entries[b].
- * workspace: hca_attend_workspace_size() bytes.
+ * workspace: hca_attend_workspace_size() bytes (currently 0).
  * --------------------------------------------------------------------- */
 size_t hca_attend_workspace_size(int Q, int H_q, int c, int64_t ldE, int n_win);
 csa_status hca_attend(const csa_geom* g, csa_dtype q_dtype, csa_dtype kv_dtype, const void* q,

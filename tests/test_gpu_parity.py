@@ -342,6 +342,52 @@ def test_csa_attend_tensor_core_paths(orc, Q, k, hole):
     assert max_abs(host(O), want) <= TOL["bf16"]
 
 
+def test_csa_attend_batch_invariance(orc):
+    """A query's output does not depend on the batch it is in: alone, inside
+    a batch of 32 and inside a permuted batch it gives the same bits."""
+    Q, Hq, c, r, N, k = 32, 64, 512, 64, 1500, 1024
+    q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(orc, Q, Hq, c, r, 4, N, k, "bf16",
+                                                            seed=41, hole=0.02)
+    g = csa.geom(c=c, rope_dims=r)
+    dE, dwin, dsink, dgain, dne = dev(E, "bf16"), dev(win, "bf16"), dev(sink, "f32"), dev(gain, "f32"), dev_i(ne)
+
+    def run(sel):
+        return host(csa.attend(dev(q[sel], "bf16"), dsink, dE, dev_i(idx[sel], torch.int32), dwin,
+                               dev_i(seq[sel], torch.int32), dev_i(pos[sel]), dne, g, q_gain=dgain))
+
+    full = run(np.arange(Q))
+    perm = np.random.default_rng(3).permutation(Q)
+    np.testing.assert_array_equal(run(perm), full[perm])
+    for i in (0, 5, 31):
+        np.testing.assert_array_equal(run(np.array([i]))[0], full[i])
+    want = orc.attend(q, sink, E, win, seq, pos, ne, rope_dims=r, idx=idx, q_gain=gain)
+    assert max_abs(full, want) <= TOL["bf16"]
+
+
+def test_csa_attend_rescale_across_tiles(orc):
+    """Window rows four times larger than the selected entries: the logits of
+    the last key tiles exceed the running reference by far, so the output
+    accumulated over the earlier tiles is rescaled part-way.
+
+    Outputs here reach about 9, where one BF16 output ulp is already 0.06 and
+    logits of standard deviation 4 magnify the BF16 rounding of Qhat and of
+    the weights in proportion. The bar is the BF16 bar scaled to the output
+    magnitude; a missed or wrong rescale errs by the size of the output."""
+    Q, Hq, c, r, N, k = 6, 64, 512, 64, 1500, 512
+    q, E, win, sink, gain, seq, ne, pos, idx = _attend_case(orc, Q, Hq, c, r, 2, N, k, "bf16",
+                                                            seed=43, hole=0.0)
+    pos[:] = 4 * N - 1  # every query sees a full selection and a full window
+    nv = np.array([orc.visible_entries(p, 4, 1, ne[s]) for p, s in zip(pos, seq)])
+    idx = synth.random_topk_indices(np.random.default_rng(44), nv, k, hole_frac=0.0)
+    win = win * 4.0  # exact in BF16
+    g = csa.geom(c=c, rope_dims=r)
+    O = csa.attend(dev(q, "bf16"), dev(sink, "f32"), dev(E, "bf16"), dev_i(idx, torch.int32),
+                   dev(win, "bf16"), dev_i(seq, torch.int32), dev_i(pos), dev_i(ne), g,
+                   q_gain=dev(gain, "f32"))
+    want = orc.attend(q, sink, E, win, seq, pos, ne, rope_dims=r, idx=idx, q_gain=gain)
+    assert max_abs(host(O), want) <= TOL["bf16"] * max(1.0, float(np.abs(want).max()))
+
+
 @pytest.mark.parametrize("Q", [24, 300])
 def test_hca_attend_tensor_core_paths(orc, Q):
     Hq, c, r, N, m = 64, 512, 64, 40, 128
