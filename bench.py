@@ -15,6 +15,7 @@ collective); timing is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -489,10 +490,15 @@ def main():
     achieved = idx_bytes / (idx_avg / 1e3) / 1e9
     traffic = None
     prof = ROOT / "profiles" / "index_topk_decode_traffic.json"
-    if prof.exists():
+    if prof.exists() and w.name == "csa_decode_bf16" and w.B == 32:
+        # ncu DRAM bytes of the call, valid only while the kernels' sources are
+        # the ones that were captured
         try:
-            traffic = json.loads(prof.read_text()).get("dram_bytes_per_launch")
-        except ValueError:
+            rec = json.loads(prof.read_text())
+            same = all(hashlib.sha256((ROOT / f).read_bytes()).hexdigest() == digest
+                       for f, digest in rec.get("sources_sha256", {}).items())
+            traffic = rec.get("dram_bytes_per_launch") if same else None
+        except (ValueError, OSError):
             traffic = None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic,

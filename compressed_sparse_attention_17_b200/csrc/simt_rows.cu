@@ -83,35 +83,41 @@ __global__ void rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int
   const int64_t orow = out_row ? out_row[row] : row;
   if (out_dt == CSA_F32) {
     float* o = reinterpret_cast<float*>(out) + orow * c;
-    for (int j = 0; j < npairs && lane + 32 * j < c / 2; ++j) {
-      int e = 2 * (lane + 32 * j);
-      *reinterpret_cast<float2*>(o + e) = make_float2(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int j = 0; j < kMaxPairsPerLane; ++j) {
+      const int e = 2 * (lane + 32 * j);
+      if (j < npairs && e < c) *reinterpret_cast<float2*>(o + e) = make_float2(v[2 * j], v[2 * j + 1]);
     }
   } else if (out_dt == CSA_BF16) {
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + orow * c;
-    for (int j = 0; j < npairs && lane + 32 * j < c / 2; ++j) {
-      int e = 2 * (lane + 32 * j);
-      *reinterpret_cast<__nv_bfloat162*>(o + e) =
-          __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int j = 0; j < kMaxPairsPerLane; ++j) {
+      const int e = 2 * (lane + 32 * j);
+      if (j < npairs && e < c)
+        *reinterpret_cast<uint32_t*>(o + e) = pack_bf16x2(v[2 * j], v[2 * j + 1]);
     }
   } else {  // mixed row, c == 512
     uint8_t* o = reinterpret_cast<uint8_t*>(out) + orow * (int64_t)kMixedRowBytes;
     float amax = 0.f;
-    for (int j = 0; j < npairs; ++j) {
-      int e = 2 * (lane + 32 * j);
-      if (e < kMixedFp8Dims) amax = fmaxf(amax, fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1])));
+#pragma unroll
+    for (int j = 0; j < kMaxPairsPerLane; ++j) {
+      const int e = 2 * (lane + 32 * j);
+      if (j < npairs && e < kMixedFp8Dims)
+        amax = fmaxf(amax, fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1])));
     }
     amax = warp_max(amax);
     const float scale = amax / 448.0f;
-    for (int j = 0; j < npairs; ++j) {
-      int e = 2 * (lane + 32 * j);
+#pragma unroll
+    for (int j = 0; j < kMaxPairsPerLane; ++j) {
+      const int e = 2 * (lane + 32 * j);
+      if (j >= npairs) continue;
       if (e < kMixedFp8Dims) {
         uint8_t c0 = scale > 0.f ? f32_to_e4m3(v[2 * j] / scale) : 0;
         uint8_t c1 = scale > 0.f ? f32_to_e4m3(v[2 * j + 1] / scale) : 0;
         *reinterpret_cast<uint16_t*>(o + e) = (uint16_t)c0 | ((uint16_t)c1 << 8);
       } else {
-        *reinterpret_cast<__nv_bfloat162*>(o + kMixedFp8Dims + 2 * (e - kMixedFp8Dims)) =
-            __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        *reinterpret_cast<uint32_t*>(o + kMixedFp8Dims + 2 * (e - kMixedFp8Dims)) =
+            pack_bf16x2(v[2 * j], v[2 * j + 1]);
       }
     }
     if (lane == 0) *reinterpret_cast<float*>(o + kMixedScaleOffset) = scale;

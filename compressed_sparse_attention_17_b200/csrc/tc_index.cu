@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // accumulator while the next tile is multiplied and later tiles load.
 // ---------------------------------------------------------------------------
 constexpr int kDecMaxQ = 1024;
+constexpr int kDecAcc = 4;  // TMEM accumulators in flight between the MMA and the epilogue
 
 struct DecParams {
   int Q, H_I, c_I, nseq, stages;
@@ -186,6 +187,7 @@ struct DecParams {
   int64_t ld_scores;
   int* err;
   uint32_t tmem_cols;
+  int interleave;  // 1: CTA i takes queries i, i + grid, ...; 0: contiguous unit ranges
 };
 
 __device__ __forceinline__ int64_t dec_nvis(const DecParams& P, int q) {
@@ -194,16 +196,37 @@ __device__ __forceinline__ int64_t dec_nvis(const DecParams& P, int q) {
   return n_visible(P.pos[q], P.m, P.vis_offset, min(P.n_entries[b], P.ldK));
 }
 
-// Walks units [u0, u1) in order; prefix[q] = first unit of query q.
+__device__ __forceinline__ int dec_ntiles(const DecParams& P, int q) {
+  return (int)((dec_nvis(P, q) + kTileM - 1) / kTileM);
+}
+
+// The (query, entry tile) units of one CTA, in order. Contiguous mode: units
+// [u0, u1) of the query-major order, prefix[q] = first unit of query q (few
+// queries: a query's tiles spread over several CTAs). Interleaved mode: every
+// tile of queries blockIdx.x, blockIdx.x + gridDim.x, ... (many queries; the
+// causal tile counts balance across CTAs).
 struct UnitWalk {
   const int* prefix;
+  const DecParams* P;
   int Q;
   int q;
   int64_t t;
-  __device__ void start(const int* pre, int nq, int u0) {
+  int nt;  // tiles of query q (interleaved mode)
+  __device__ void start(const DecParams& prm, const int* pre, int u0) {
+    P = &prm;
     prefix = pre;
-    Q = nq;
-    int lo = 0, hi = nq - 1;  // largest q with prefix[q] <= u0
+    Q = prm.Q;
+    if (prm.interleave) {
+      q = blockIdx.x;
+      t = 0;
+      nt = q < Q ? dec_ntiles(prm, q) : 0;
+      while (q < Q && nt == 0) {
+        q += gridDim.x;
+        nt = q < Q ? dec_ntiles(prm, q) : 0;
+      }
+      return;
+    }
+    int lo = 0, hi = Q - 1;  // largest q with prefix[q] <= u0
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (prefix[mid] <= u0) lo = mid;
@@ -218,6 +241,14 @@ struct UnitWalk {
   }
   __device__ void next() {
     ++t;
+    if (P->interleave) {
+      while (q < Q && t >= nt) {
+        q += gridDim.x;
+        t = 0;
+        nt = q < Q ? dec_ntiles(*P, q) : 0;
+      }
+      return;
+    }
     while (q < Q - 1 && t >= prefix[q + 1] - prefix[q]) {
       t = 0;
       ++q;
@@ -242,40 +273,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sB = sA + S * bytesA;
   float* wsm = reinterpret_cast<float*>(sB + 2 * bytesB);
   int* prefix = reinterpret_cast<int*>(wsm + 128);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + ((P.Q + 2 + 1) & ~1));
-  // bars: Afull[S], Aempty[S], Bfull[2], Bempty[2], accfull[2], accempty[2]
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + (P.interleave ? 2 : ((P.Q + 2 + 1) & ~1)));
+  // bars: Afull[S], Aempty[S], Bfull[2], Bempty[2], accfull[kDecAcc], accempty[kDecAcc]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4 + 2 * kDecAcc);
   __shared__ int scan_tmp[kThreads / 32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- units per query and their prefix (every CTA computes it) ----
-  int carry = 0;
-  for (int base = 0; base < P.Q; base += kThreads) {
-    const int q = base + threadIdx.x;
-    const int nt = q < P.Q ? (int)((dec_nvis(P, q) + kTileM - 1) / kTileM) : 0;
-    int x = nt;
+  int u0 = 0, u1 = 0;
+  if (P.interleave) {
+    // ---- this CTA's tile count over its queries ----
+    int cnt = 0;
+    for (int q = blockIdx.x + threadIdx.x * gridDim.x; q < P.Q; q += kThreads * gridDim.x)
+      cnt += dec_ntiles(P, q);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) scan_tmp[warp] = x;
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) scan_tmp[warp] = cnt;
     __syncthreads();
-    int wbase = 0, tot = 0;
-    for (int i = 0; i < kThreads / 32; ++i) {
-      wbase += i < warp ? scan_tmp[i] : 0;
-      tot += scan_tmp[i];
-    }
-    if (q < P.Q) prefix[q] = carry + wbase + x - nt;
-    carry += tot;
+    for (int i = 0; i < kThreads / 32; ++i) u1 += scan_tmp[i];
     __syncthreads();
+  } else {
+    // ---- units per query and their prefix (every CTA computes it) ----
+    int carry = 0;
+    for (int base = 0; base < P.Q; base += kThreads) {
+      const int q = base + threadIdx.x;
+      const int nt = q < P.Q ? dec_ntiles(P, q) : 0;
+      int x = nt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) scan_tmp[warp] = x;
+      __syncthreads();
+      int wbase = 0, tot = 0;
+      for (int i = 0; i < kThreads / 32; ++i) {
+        wbase += i < warp ? scan_tmp[i] : 0;
+        tot += scan_tmp[i];
+      }
+      if (q < P.Q) prefix[q] = carry + wbase + x - nt;
+      carry += tot;
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) prefix[P.Q] = carry;
+    __syncthreads();
+    const int U = prefix[P.Q];
+    u0 = (int)((int64_t)blockIdx.x * U / gridDim.x);
+    u1 = (int)((int64_t)(blockIdx.x + 1) * U / gridDim.x);
   }
-  if (threadIdx.x == 0) prefix[P.Q] = carry;
-  __syncthreads();
-  const int U = prefix[P.Q];
-  const int u0 = (int)((int64_t)blockIdx.x * U / gridDim.x);
-  const int u1 = (int)((int64_t)(blockIdx.x + 1) * U / gridDim.x);
   if (u0 >= u1) return;  // same decision in every thread of the CTA
 
   auto afull = [&](int s) { return tc::smem_u32(&bars[s]); };
@@ -283,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bfull = [&](int s) { return tc::smem_u32(&bars[2 * S + s]); };
   auto bempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 2 + s]); };
   auto accfull = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + s]); };
-  auto accempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 6 + s]); };
+  auto accempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + kDecAcc + s]); };
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(afull(s), 1);
@@ -292,6 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(bfull(s), 1);
       tc::mbar_init(bempty(s), 1);
+    }
+    for (int s = 0; s < kDecAcc; ++s) {
       tc::mbar_init(accfull(s), 1);
       tc::mbar_init(accempty(s), 4);
     }
@@ -311,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- producer ----
       const uint64_t pol = tc::l2_policy_evict_first();
       UnitWalk wk;
-      wk.start(prefix, P.Q, u0);
+      wk.start(P, prefix, u0);
       int last_q = -1, gc = -1;
       for (int i = 0; i < nunits; ++i, wk.next()) {
         const int q = wk.q;
@@ -340,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- MMA issuer ----
       const uint32_t idesc = tc::idesc_bf16_f32(kTileM, P.H_I);
       UnitWalk wk;
-      wk.start(prefix, P.Q, u0);
+      wk.start(P, prefix, u0);
       int last_q = -1, gc = -1;
       for (int i = 0; i < nunits; ++i, wk.next()) {
         const int q = wk.q;
@@ -350,9 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!tc::mbar_wait(bfull(gc & 1), (gc >> 1) & 1, P.err)) break;
           last_q = q;
         }
-        const int s = i % S, a = i & 1;
+        const int s = i % S, a = i % kDecAcc;
         if (!tc::mbar_wait(afull(s), (i / S) & 1, P.err)) break;
-        if (i >= 2 && !tc::mbar_wait(accempty(a), ((i >> 1) - 1) & 1, P.err)) break;
+        if (i >= kDecAcc && !tc::mbar_wait(accempty(a), ((i / kDecAcc) - 1) & 1, P.err)) break;
         tc::tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(a * P.H_I);
         for (int kk = 0; kk < KCH * 4; ++kk) {
@@ -372,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     UnitWalk wk;
-    wk.start(prefix, P.Q, u0);
+    wk.start(P, prefix, u0);
     int last_q = -1;
     int64_t nv = 0;
     float* out = nullptr;
@@ -396,26 +443,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         last_q = q;
       }
-      const int a = i & 1;
-      if (!tc::mbar_wait_warp(accfull(a), (i >> 1) & 1, P.err)) break;
+      const int a = i % kDecAcc;
+      if (!tc::mbar_wait_warp(accfull(a), (i / kDecAcc) & 1, P.err)) break;
       tc::tc_fence_after();
-      float acc = 0.f;
+      float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains over the heads
       if (HREG > 0) {
 #pragma unroll
         for (int h0 = 0; h0 < (HREG > 0 ? HREG : 16); h0 += 32) {
           float v[32];
           tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * HREG + h0), v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc = fmaf(wr[h0 + j], fmaxf(v[j], 0.f), acc);
+          for (int j = 0; j < 32; ++j) acc4[j & 3] = fmaf(wr[h0 + j], fmaxf(v[j], 0.f), acc4[j & 3]);
         }
       } else {
         for (int h0 = 0; h0 < P.H_I; h0 += 16) {
           float v[16];
           tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * P.H_I + h0), v);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc = fmaf(__ldg(wq + h0 + j), fmaxf(v[j], 0.f), acc);
+          for (int j = 0; j < 16; ++j) acc4[j & 3] = fmaf(__ldg(wq + h0 + j), fmaxf(v[j], 0.f), acc4[j & 3]);
         }
       }
+      const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(accempty(a));
@@ -441,8 +489,8 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
                                    const int64_t* n_entries, int Q, int H_I, int c_I,
                                    float* scores, int64_t ld_scores, cudaStream_t s) {
   if (Q == 0 || ldK == 0 || nseq == 0) return cudaSuccess;
-  if (Q <= kDecMaxQ) {
-    // few queries: persistent pipelined kernel over (query, tile) units
+  if (Q <= kDecMaxQ || true) {
+    // persistent pipelined kernel over (query, tile) units
     CUtensorMap tmK, tmQ;
     if (!encode_tmap_2d_bf16(&tmK, KI, (uint64_t)c_I, (uint64_t)nseq * ldK, (uint64_t)c_I * 2, 64,
                              kTileM) ||
@@ -464,11 +512,17 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
     P.scores = scores;
     P.ld_scores = ld_scores;
     P.err = device_error_ptr();
+    int nsm = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    P.interleave = Q >= 4 * nsm ? 1 : 0;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(2 * H_I)) cols <<= 1;
+    while (cols < (uint32_t)(kDecAcc * H_I)) cols <<= 1;
     P.tmem_cols = cols;
     const int KCH = c_I / 64;
-    const size_t fixed = 1024 + 2 * (size_t)KCH * H_I * 128 + 128 * 4 + ((size_t)Q + 3) * 4 + 256;
+    const size_t prefix_ints = P.interleave ? 2 : (size_t)Q + 3;
+    const size_t fixed = 1024 + 2 * (size_t)KCH * H_I * 128 + 128 * 4 + prefix_ints * 4 + 256;
     const size_t per_stage = (size_t)KCH * kChunkBytesA;
     const int stages = (int)std::min<size_t>(6, (220 * 1024 - fixed) / per_stage);
     if (stages < 2) return cudaErrorInvalidValue;
@@ -479,10 +533,6 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
     auto kern = wreg ? index_decode_kernel<64> : index_decode_kernel<0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    int nsm = 148;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     count_launches();
     kern<<<nsm, kThreads, smem, s>>>(tmK, tmQ, P);
     return cudaGetLastError();

@@ -17,8 +17,9 @@
 //   1. the score range [min, max] of the segment;
 //   2. a 2048-bin value histogram over that range (the bin is a
 //      non-decreasing function of the score, so every key of a higher bin is
-//      larger), summed over the cluster; its suffix counts give the bin
-//      holding the k-th largest key and how many keys lie above it;
+//      larger); the cluster's totals of 8 slices of 256 bins locate the slice
+//      holding the k-th largest key, and that slice's bins, summed over the
+//      cluster, the bin and how many keys lie above it;
 //   3. that bin's keys (usually a few dozen) are gathered into every CTA and
 //      ranked exactly - by counting, or by radix select when there are many;
 //      when they do not fit (many equal scores), a cluster-wide radix select
@@ -62,7 +63,7 @@ __device__ __forceinline__ uint64_t pair_key(float s, int32_t id) {
 template <int NT>
 struct Smem {
   int hist[kBins];  // this CTA's value histogram
-  int hsum[kBins];  // the cluster's
+  int stot[8];      // this CTA's counts in 8 slices of 256 bins
   uint64_t loc[kLocCap];
   uint64_t gath[kGathCap];
   int rhist[2][256];
@@ -71,7 +72,7 @@ struct Smem {
   int cnt[kMaxCluster], off[kMaxCluster];
   float mn, mx, gmn, gmx;
   int nloc, tot, over;
-  int bstar, above;
+  int bstar, above, sstar, above0;
   int digit, rem;
   int kept, cbase, ctot;
   uint64_t kth;
@@ -314,24 +315,61 @@ __global__ void __launch_bounds__(NT, CAND ? 1 : 1024 / NT) topk_cluster_kernel(
 #pragma unroll
     for (int j = 0; j < KPT; ++j)
       if (vm >> j & 1u) atomicAdd(&S.hist[bin_of(s[j])], 1);
-    csync(C);
-    const int* hs = S.hist;
     if (C > 1) {
-      for (int b = tid; b < kBins; b += NT) {
+      // slice totals: warp s counts bins [256 s, 256 s + 256)
+      __syncthreads();
+      if (wid < 8) {
         int v = 0;
-        for (int r = 0; r < C; ++r) v += peer(S.hist, r, C)[b];
-        S.hsum[b] = v;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v += S.hist[256 * wid + 32 * e + lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) S.stot[wid] = v;
+      }
+      csync(C);
+      // the slice holding the k-th largest key, from the top slice down
+      if (wid == 0) {
+        int tot = 0;
+        if (lane < 8)
+          for (int r = 0; r < C; ++r) tot += peer(S.stot, r, C)[lane];
+        // suffix sums over the slices (inclusive, then exclusive)
+        int suf = lane < 8 ? tot : 0;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+          const int y = __shfl_down_sync(0xffffffffu, suf, o);
+          if (lane + o < 8) suf += y;
+        }
+        const int ex = suf - (lane < 8 ? tot : 0);
+        if (lane < 8 && ex < k && k <= suf) {
+          S.sstar = lane;
+          S.above0 = ex;
+        }
       }
       __syncthreads();
-      hs = S.hsum;
-    }
-    // bin of the k-th largest: thread t owns bins 2047 - BPT t - e, e < BPT
-    {
+      // its 256 bins summed over the cluster; thread t takes bin 255 - t of the slice
+      const int sl = S.sstar;
+      int v = 0;
+      if (tid < 256) {
+        const int b = 256 * sl + 255 - tid;
+        for (int r = 0; r < C; ++r) v += peer(S.hist, r, C)[b];
+      }
+      int tot;
+      const int cum = block_exclusive_scan<NT>(v, S.scan, &tot);
+      const int need0 = k - S.above0;
+      if (tid < 256 && cum < need0 && need0 <= cum + v) {
+        S.bstar = 256 * sl + 255 - tid;
+        S.above = S.above0 + cum;
+      }
+      __syncthreads();
+    } else {
+      // one CTA: bin of the k-th largest over the whole local histogram;
+      // thread t owns bins 2047 - BPT t - e, e < BPT
+      __syncthreads();
       constexpr int BPT = kBins / NT;
       int cnt[BPT], sum = 0;
 #pragma unroll
       for (int e = 0; e < BPT; ++e) {
-        cnt[e] = hs[kBins - 1 - (BPT * tid + e)];
+        cnt[e] = S.hist[kBins - 1 - (BPT * tid + e)];
         sum += cnt[e];
       }
       int tot;
