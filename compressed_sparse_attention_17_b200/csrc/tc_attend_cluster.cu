@@ -264,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       //      of chunk l / 4); four heads at a time ----
       float gn[16];
       float2 rt[8];  // (cos, sin) of each pair of this lane, (1, 0) outside the rotated dims
+      float qscale = 1.f;  // RMSNorm factor of head h when it is applied to the logits
 #pragma unroll
       for (int i = 0; i < 16; ++i) gn[i] = P.q_gain ? P.q_gain[16 * lane + i] : 1.f;
 #pragma unroll
@@ -274,56 +275,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!tc::mbar_wait_warp(bar(kQRaw), 0, P.err)) flags[0] = 1;
       uint8_t* qch = sm + kOffQ + (lane >> 2) * 8192;
       const uint32_t g0 = (uint32_t)((2 * lane) & 7);
-      for (int j0 = 0; j0 < 16; j0 += 4) {
-        uint4* ptr[4][2];
-        uint4 raw[4][2];
-        float ss[4];
+      if (P.q_gain == nullptr) {
+        // Without a gain, RMSNorm scales each head by one factor, applied to
+        // its logits instead: only the rotated dims change here, in place,
+        // and the MMA starts as soon as they are written.
+        if (16 * lane + 16 > kDim - P.r) {
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t hh = (uint32_t)(16 * warp + j);
+            uint4* p0 = reinterpret_cast<uint4*>(qch + tc::sw128_offset(hh, g0));
+            uint4* p1 = reinterpret_cast<uint4*>(qch + tc::sw128_offset(hh, g0 + 1));
+            const uint4 r0 = *p0, r1 = *p1;
+            const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            uint32_t o[8];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const uint32_t hh = (uint32_t)(16 * warp + j0 + jj);
-          ptr[jj][0] = reinterpret_cast<uint4*>(qch + tc::sw128_offset(hh, g0));
-          ptr[jj][1] = reinterpret_cast<uint4*>(qch + tc::sw128_offset(hh, g0 + 1));
-          raw[jj][0] = *ptr[jj][0];
-          raw[jj][1] = *ptr[jj][1];
-        }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const uint32_t w[8] = {raw[jj][0].x, raw[jj][0].y, raw[jj][0].z, raw[jj][0].w,
-                                 raw[jj][1].x, raw[jj][1].y, raw[jj][1].z, raw[jj][1].w};
-          float s2 = 0.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
-            s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
+            for (int i = 0; i < 8; ++i) {
+              const float a = bf16_lo(w[i]), bb = bf16_hi(w[i]);
+              o[i] = pack_bf16x2(a * rt[i].x - bb * rt[i].y, a * rt[i].y + bb * rt[i].x);
+            }
+            *p0 = make_uint4(o[0], o[1], o[2], o[3]);
+            *p1 = make_uint4(o[4], o[5], o[6], o[7]);
           }
-          ss[jj] = s2;
         }
+        __syncwarp();  // the rotated dims are read back below by every lane
+        tc::fence_proxy_async();
+        tc::mbar_arrive(bar(kQReady));
+        // RMSNorm factors of this warp's heads (the rotation keeps the sum
+        // of squares); lanes l and l + 16 keep head 16 w + l % 16's
+        for (int j0 = 0; j0 < 16; j0 += 4) {
+          float ss[4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t hh = (uint32_t)(16 * warp + j0 + jj);
+            const uint4 r0 = *reinterpret_cast<const uint4*>(qch + tc::sw128_offset(hh, g0));
+            const uint4 r1 = *reinterpret_cast<const uint4*>(qch + tc::sw128_offset(hh, g0 + 1));
+            const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            float s2 = 0.f;
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) ss[jj] += __shfl_xor_sync(0xffffffffu, ss[jj], o);
-        }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const float inv = rsqrtf(ss[jj] * (1.f / (float)kDim) + P.eps);
-          const uint32_t w[8] = {raw[jj][0].x, raw[jj][0].y, raw[jj][0].z, raw[jj][0].w,
-                                 raw[jj][1].x, raw[jj][1].y, raw[jj][1].z, raw[jj][1].w};
-          uint32_t o[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float a = bf16_lo(w[i]) * inv * gn[2 * i];
-            const float bb = bf16_hi(w[i]) * inv * gn[2 * i + 1];
-            o[i] = pack_bf16x2(a * rt[i].x - bb * rt[i].y, a * rt[i].y + bb * rt[i].x);
+            for (int i = 0; i < 8; ++i) {
+              const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+              s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
+            }
+            ss[jj] = s2;
           }
-          *ptr[jj][0] = make_uint4(o[0], o[1], o[2], o[3]);
-          *ptr[jj][1] = make_uint4(o[4], o[5], o[6], o[7]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) ss[jj] += __shfl_xor_sync(0xffffffffu, ss[jj], o);
+          }
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            if ((lane & 15) == j0 + jj) qscale = rsqrtf(ss[jj] * (1.f / (float)kDim) + P.eps);
         }
+      } else {
+        for (int j0 = 0; j0 < 16; j0 += 4) {
+          uint4* ptr[4][2];
+          uint4 raw[4][2];
+          float ss[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t hh = (uint32_t)(16 * warp + j0 + jj);
+            ptr[jj][0] = reinterpret_cast<uint4*>(qch + tc::sw128_offset(hh, g0));
+            ptr[jj][1] = reinterpret_cast<uint4*>(qch + tc::sw128_offset(hh, g0 + 1));
+            raw[jj][0] = *ptr[jj][0];
+            raw[jj][1] = *ptr[jj][1];
+          }
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t w[8] = {raw[jj][0].x, raw[jj][0].y, raw[jj][0].z, raw[jj][0].w,
+                                   raw[jj][1].x, raw[jj][1].y, raw[jj][1].z, raw[jj][1].w};
+            float s2 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+              s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
+            }
+            ss[jj] = s2;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) ss[jj] += __shfl_xor_sync(0xffffffffu, ss[jj], o);
+          }
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const float inv = rsqrtf(ss[jj] * (1.f / (float)kDim) + P.eps);
+            const uint32_t w[8] = {raw[jj][0].x, raw[jj][0].y, raw[jj][0].z, raw[jj][0].w,
+                                   raw[jj][1].x, raw[jj][1].y, raw[jj][1].z, raw[jj][1].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float a = bf16_lo(w[i]) * inv * gn[2 * i];
+              const float bb = bf16_hi(w[i]) * inv * gn[2 * i + 1];
+              o[i] = pack_bf16x2(a * rt[i].x - bb * rt[i].y, a * rt[i].y + bb * rt[i].x);
+            }
+            *ptr[jj][0] = make_uint4(o[0], o[1], o[2], o[3]);
+            *ptr[jj][1] = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+        }
+        tc::fence_proxy_async();
+        tc::mbar_arrive(bar(kQReady));
       }
-      tc::fence_proxy_async();
-      tc::mbar_arrive(bar(kQReady));
 
       // ---- softmax over this CTA's tiles ----
-      const float scale2 = kLog2e / sqrtf((float)kDim);
+      const float sc = kLog2e / sqrtf((float)kDim) * qscale;
       const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
       for (int t = 0; t < T; ++t) {
         const int buf = t & 1;
@@ -339,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          s[i] = i < nvalid ? s[i] * scale2 : -INFINITY;
+          s[i] = i < nvalid ? s[i] * sc : -INFINITY;
           m8[i & 7] = fmaxf(m8[i & 7], s[i]);
         }
         const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
