@@ -247,15 +247,27 @@ class Prefill:
         torch.cuda.synchronize(device)
         log(f"[prefill] setup {time.time() - t0:.1f}s: T={T}")
 
-    def step(self):
+    def index_flops(self):
+        """Algorithmic FLOPs of the prefill indexer: 2 H_I c_I per visible
+        (query, entry) pair, entry s visible to token t when s < (t + 1) / m."""
+        w = self.w
+        t = np.arange(w.T, dtype=np.int64)
+        nvis = np.minimum((t + self.g.vis_offset) // w.m, w.T // w.m)
+        return int(nvis.sum()) * 2 * w.H_I * w.c_I
+
+    def step(self, ev=None):
         t, w = self.t, self.w
         E = csa.compress(t["H"], t["W_aKV"], t["W_aZ"], t["bias"], self.g, W_bKV=t["W_bKV"],
                          W_bZ=t["W_bZ"])
         KI = csa.compress(t["H"], t["WI_aKV"], t["WI_aZ"], t["biasI"], self.gI, W_bKV=t["WI_bKV"],
                           W_bZ=t["WI_bZ"])
         win = csa.rmsnorm_rope(t["kv_win"], self.g, pos0=0, pos_step=1)
+        if ev:
+            ev[0].record()
         csa.index_topk(t["qI"], t["w"], KI[None], self.seq, self.pos, self.ne, w.k, self.g,
                        out=self.idx)
+        if ev:
+            ev[1].record()
         csa.attend(t["q"], t["sink"], E[None], self.idx, win[None], self.seq, self.pos, self.ne,
                    self.g, out=self.O)
 
@@ -513,12 +525,25 @@ def main():
         torch.cuda.empty_cache()
         pw = synth.WORKLOADS[args.prefill_workload]()
         pre = (Prefill if pw.kind == "csa_prefill" else HcaPrefill)(pw, device)
-        pms, _ = time_steps(lambda ev: pre.step(), max(3, args.steps // 4), 3, device, flush)
+        csa_pre = pw.kind == "csa_prefill"
+        pms, ims = time_steps(lambda ev: pre.step(ev), max(3, args.steps // 4), 3, device, flush,
+                              extra_events=2 if csa_pre else 0)
         pms_max = max_over_ranks(statistics.mean(pms))
         prefill = {"metric": ("CSA" if pw.kind == "csa_prefill" else "HCA") + " prefill tokens/s",
                    "value": args.gpus * pw.T / (pms_max / 1e3),
                    "unit": "tokens/s", "ms_per_step": pms_max,
                    "config": {"workload": pw.name, "T": pw.T, "d": pw.d, "top_k": pw.k}}
+        if csa_pre:
+            # tensor roofline of the indexer: the whole csa_index_topk call
+            # (score launch + top-k launch) against the indexer's FLOPs alone
+            ims_max = max_over_ranks(statistics.mean(ims))
+            fl = pre.index_flops()
+            ach = fl / (ims_max / 1e3) / 1e12
+            prefill["indexer_roofline"] = {
+                "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
+                "frac": ach / tflops, "kernel": "csa_index_topk (prefill, indexer + top-k launches)",
+                "kernel_ms": ims_max, "algorithmic_flop": fl,
+                "peak_source": f"{peak_kind} dense BF16 GEMM (burst)"}
         del pre
 
     clk.__exit__(None, None, None)

@@ -12,8 +12,9 @@
 // ReLU, the head weights and the head sum in registers, so each thread owns
 // one entry and no cross-thread reduction is needed.
 //
-// Warp roles (192 threads): warp 0 issues the TMA loads, warp 1 owns the
-// TMEM allocation and issues the MMAs, warps 2-5 run the epilogue.
+// Warp roles: warp 0 issues the TMA loads, warp 1 owns the TMEM allocation
+// and issues the MMAs, the remaining warps (4, or 8 for query groups) run the
+// epilogue.
 #include <algorithm>
 
 #include "internal.h"
@@ -23,24 +24,39 @@ namespace csa {
 
 namespace {
 
-constexpr int kThreads = 192;
 constexpr int kTileM = 128;
 constexpr int kChunkBytesA = kTileM * 128;  // 128 rows x 64 BF16
 
 // ---------------------------------------------------------------------------
-// Persistent, pipelined kernel (one CTA per SM) over (query, 128-entry tile)
-// units: with few queries (decode) every CTA takes a balanced contiguous
-// range of units, which may span query boundaries; with many (prefill) CTA i
-// takes every tile of queries i, i + grid, ... Warp 0 streams the key tiles
-// through a ring of shared-memory stages (TMA, evict-first L2 policy) and
-// loads a query's qI into one of two slots when the query changes; warp 1
-// issues the MMAs into one of four TMEM accumulators; warps 2-5 reduce the
-// accumulator while the next tile is multiplied and later tiles load.
+// Persistent, pipelined kernel (one CTA per SM) over (query group, 128-entry
+// tile) units. A group is G consecutive queries of one sequence: its G x H_I
+// (query, head) rows form the MMA's N dimension, so one key tile serves the
+// whole group (G = 4 for long single-sequence runs such as prefill, where the
+// same keys are read by every query; G = 1 otherwise). With few groups every
+// CTA takes a balanced contiguous range of units, which may span group
+// boundaries; with many, CTA i takes every tile of groups i, i + grid, ...
+// Warp 0 streams the key tiles through a ring of shared-memory stages (TMA,
+// evict-first L2 policy) and loads a group's qI into one of two slots when
+// the group changes; warp 1 issues the MMAs into one of the TMEM accumulators;
+// warps 2-5 reduce an accumulator while the next tile is multiplied and later
+// tiles load.
 // ---------------------------------------------------------------------------
-constexpr int kDecAcc = 4;  // TMEM accumulators in flight between the MMA and the epilogue
+constexpr int kDecAcc = 4;  // G = 1: TMEM accumulators in flight between the MMA and the epilogue
+constexpr int kGrpAcc = 2;  // G > 1: two accumulators of G x H_I columns
+
+// Warp roles: warp 0 loads, warp 1 issues the MMAs, the rest run the
+// epilogue (G = 1: 4 warps, one per TMEM lane quadrant; G > 1: 8 warps, two
+// per quadrant, each taking half of the group's queries).
+template <int G>
+struct GroupCfg {
+  static constexpr int acc = G == 1 ? kDecAcc : kGrpAcc;
+  static constexpr int epi_warps = G == 1 ? 4 : 8;
+  static constexpr int threads = 64 + 32 * epi_warps;
+};
 
 struct DecParams {
   int Q, H_I, c_I, nseq, stages;
+  int NG;  // query groups of G consecutive queries
   int64_t ldK;
   int m, vis_offset;
   const int32_t* seq_of_q;
@@ -64,11 +80,24 @@ __device__ __forceinline__ int dec_ntiles(const DecParams& P, int q) {
   return (int)((dec_nvis(P, q) + kTileM - 1) / kTileM);
 }
 
-// The (query, entry tile) units of one CTA, in order. Contiguous mode: units
-// [u0, u1) of the query-major order, prefix[q] = first unit of query q (few
-// queries: a query's tiles spread over several CTAs). Interleaved mode: every
-// tile of queries blockIdx.x, blockIdx.x + gridDim.x, ... (many queries; the
-// causal tile counts balance across CTAs).
+// Entry tiles of group g: those of its member that sees the most entries.
+template <int G>
+__device__ __forceinline__ int grp_ntiles(const DecParams& P, int g) {
+  int nt = 0;
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    const int q = g * G + j;
+    if (q < P.Q) nt = max(nt, dec_ntiles(P, q));
+  }
+  return nt;
+}
+
+// The (group, entry tile) units of one CTA, in order. Contiguous mode: units
+// [u0, u1) of the group-major order, prefix[g] = first unit of group g (few
+// groups: a group's tiles spread over several CTAs). Interleaved mode: every
+// tile of groups blockIdx.x, blockIdx.x + gridDim.x, ... (many groups; the
+// causal tile counts balance across CTAs). q below is the group index.
+template <int G>
 struct UnitWalk {
   const int* prefix;
   const DecParams* P;
@@ -79,14 +108,14 @@ struct UnitWalk {
   __device__ void start(const DecParams& prm, const int* pre, int u0) {
     P = &prm;
     prefix = pre;
-    Q = prm.Q;
+    Q = prm.NG;
     if (prm.interleave) {
       q = blockIdx.x;
       t = 0;
-      nt = q < Q ? dec_ntiles(prm, q) : 0;
+      nt = q < Q ? grp_ntiles<G>(prm, q) : 0;
       while (q < Q && nt == 0) {
         q += gridDim.x;
-        nt = q < Q ? dec_ntiles(prm, q) : 0;
+        nt = q < Q ? grp_ntiles<G>(prm, q) : 0;
       }
       return;
     }
@@ -109,7 +138,7 @@ struct UnitWalk {
       while (q < Q && t >= nt) {
         q += gridDim.x;
         t = 0;
-        nt = q < Q ? dec_ntiles(*P, q) : 0;
+        nt = q < Q ? grp_ntiles<G>(*P, q) : 0;
       }
       return;
     }
@@ -121,9 +150,10 @@ struct UnitWalk {
 };
 
 // HREG = H_I when the head weights of the current query are kept in
-// registers (reloaded when the query changes), 0 for read-through loads.
-template <int HREG>
-__global__ void __launch_bounds__(kThreads, 1)
+// registers (reloaded when the query changes; G = 1), 0 for read-through
+// loads. G = queries per group (1, or 4 with H_I = 64).
+template <int HREG, int G>
+__global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
     index_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                         DecParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -131,25 +161,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const int KCH = P.c_I / 64;
   const int S = P.stages;
+  constexpr int NACC = GroupCfg<G>::acc;
+  const int NW = G * P.H_I;  // MMA N: the group's (query, head) rows
   const int bytesA = KCH * kChunkBytesA;
-  const int bytesB = KCH * P.H_I * 128;
+  const int bytesB = KCH * NW * 128;
   uint8_t* sA = smem;
   uint8_t* sB = sA + S * bytesA;
-  float* wsm = reinterpret_cast<float*>(sB + 2 * bytesB);
-  int* prefix = reinterpret_cast<int*>(wsm + 128);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + (P.interleave ? 2 : ((P.Q + 2 + 1) & ~1)));
-  // bars: Afull[S], Aempty[S], Bfull[2], Bempty[2], accfull[kDecAcc], accempty[kDecAcc]
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4 + 2 * kDecAcc);
+  int* prefix = reinterpret_cast<int*>(sB + 2 * bytesB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + (P.interleave ? 2 : ((P.NG + 2 + 1) & ~1)));
+  // bars: Afull[S], Aempty[S], Bfull[2], Bempty[2], accfull[NACC], accempty[NACC]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4 + 2 * NACC);
+  constexpr int kThreads = GroupCfg<G>::threads;
+  constexpr int kEpi = GroupCfg<G>::epi_warps;
   __shared__ int scan_tmp[kThreads / 32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   int u0 = 0, u1 = 0;
   if (P.interleave) {
-    // ---- this CTA's tile count over its queries ----
+    // ---- this CTA's tile count over its groups ----
     int cnt = 0;
-    for (int q = blockIdx.x + threadIdx.x * gridDim.x; q < P.Q; q += kThreads * gridDim.x)
-      cnt += dec_ntiles(P, q);
+    for (int q = blockIdx.x + threadIdx.x * gridDim.x; q < P.NG; q += kThreads * gridDim.x)
+      cnt += grp_ntiles<G>(P, q);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     if (lane == 0) scan_tmp[warp] = cnt;
@@ -157,11 +190,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kThreads / 32; ++i) u1 += scan_tmp[i];
     __syncthreads();
   } else {
-    // ---- units per query and their prefix (every CTA computes it) ----
+    // ---- units per group and their prefix (every CTA computes it) ----
     int carry = 0;
-    for (int base = 0; base < P.Q; base += kThreads) {
+    for (int base = 0; base < P.NG; base += kThreads) {
       const int q = base + threadIdx.x;
-      const int nt = q < P.Q ? dec_ntiles(P, q) : 0;
+      const int nt = q < P.NG ? grp_ntiles<G>(P, q) : 0;
       int x = nt;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -175,13 +208,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         wbase += i < warp ? scan_tmp[i] : 0;
         tot += scan_tmp[i];
       }
-      if (q < P.Q) prefix[q] = carry + wbase + x - nt;
+      if (q < P.NG) prefix[q] = carry + wbase + x - nt;
       carry += tot;
       __syncthreads();
     }
-    if (threadIdx.x == 0) prefix[P.Q] = carry;
+    if (threadIdx.x == 0) prefix[P.NG] = carry;
     __syncthreads();
-    const int U = prefix[P.Q];
+    const int U = prefix[P.NG];
     u0 = (int)((int64_t)blockIdx.x * U / gridDim.x);
     u1 = (int)((int64_t)(blockIdx.x + 1) * U / gridDim.x);
   }
@@ -192,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bfull = [&](int s) { return tc::smem_u32(&bars[2 * S + s]); };
   auto bempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 2 + s]); };
   auto accfull = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + s]); };
-  auto accempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + kDecAcc + s]); };
+  auto accempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + NACC + s]); };
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(afull(s), 1);
@@ -202,9 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(bfull(s), 1);
       tc::mbar_init(bempty(s), 1);
     }
-    for (int s = 0; s < kDecAcc; ++s) {
+    for (int s = 0; s < NACC; ++s) {
       tc::mbar_init(accfull(s), 1);
-      tc::mbar_init(accempty(s), 4);
+      tc::mbar_init(accempty(s), kEpi);
     }
     tc::fence_barrier_init();
     tc::prefetch_tmap(&tmK);
@@ -221,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ---- producer ----
       const uint64_t pol = tc::l2_policy_evict_first();
-      UnitWalk wk;
+      UnitWalk<G> wk;
       wk.start(P, prefix, u0);
       int last_q = -1, gc = -1;
       for (int i = 0; i < nunits; ++i, wk.next()) {
@@ -232,14 +265,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (gc >= 2 && !tc::mbar_wait(bempty(bs), ((gc >> 1) - 1) & 1, P.err)) break;
           tc::mbar_arrive_expect_tx(bfull(bs), (uint32_t)bytesB);
           for (int ch = 0; ch < KCH; ++ch)
-            tc::tma_load_2d(tc::smem_u32(sB + bs * bytesB + ch * P.H_I * 128), &tmQ, ch * 64,
-                            q * P.H_I, bfull(bs));
+            tc::tma_load_2d(tc::smem_u32(sB + bs * bytesB + ch * NW * 128), &tmQ, ch * 64, q * NW,
+                            bfull(bs));
           last_q = q;
         }
         const int s = i % S;
         if (i >= S && !tc::mbar_wait(aempty(s), ((i / S) - 1) & 1, P.err)) break;
         tc::mbar_arrive_expect_tx(afull(s), (uint32_t)bytesA);
-        const int32_t y = (int32_t)((int64_t)P.seq_of_q[q] * P.ldK + wk.t * kTileM);
+        // groups of several queries are formed only over a single sequence
+        const int64_t seq = G == 1 ? (int64_t)P.seq_of_q[q] : 0;
+        const int32_t y = (int32_t)(seq * P.ldK + wk.t * kTileM);
         for (int ch = 0; ch < KCH; ++ch)
           tc::tma_load_2d_hint(tc::smem_u32(sA + s * bytesA + ch * kChunkBytesA), &tmK, ch * 64, y,
                                afull(s), pol);
@@ -249,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---- MMA issuer ----
-      const uint32_t idesc = tc::idesc_bf16_f32(kTileM, P.H_I);
-      UnitWalk wk;
+      const uint32_t idesc = tc::idesc_bf16_f32(kTileM, NW);
+      UnitWalk<G> wk;
       wk.start(P, prefix, u0);
       int last_q = -1, gc = -1;
       for (int i = 0; i < nunits; ++i, wk.next()) {
@@ -261,16 +296,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!tc::mbar_wait(bfull(gc & 1), (gc >> 1) & 1, P.err)) break;
           last_q = q;
         }
-        const int s = i % S, a = i % kDecAcc;
+        const int s = i % S, a = i % NACC;
         if (!tc::mbar_wait(afull(s), (i / S) & 1, P.err)) break;
-        if (i >= kDecAcc && !tc::mbar_wait(accempty(a), ((i / kDecAcc) - 1) & 1, P.err)) break;
+        if (i >= NACC && !tc::mbar_wait(accempty(a), ((i / NACC) - 1) & 1, P.err)) break;
         tc::tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(a * P.H_I);
+        const uint32_t d = tmem + (uint32_t)(a * NW);
         for (int kk = 0; kk < KCH * 4; ++kk) {
           const int ch = kk >> 2;
           const uint32_t off = (uint32_t)(kk & 3) * 32;
           tc::mma_bf16(d, tc::sdesc_kmajor_sw128(tc::smem_u32(sA + s * bytesA + ch * kChunkBytesA) + off),
-                       tc::sdesc_kmajor_sw128(tc::smem_u32(sB + (gc & 1) * bytesB + ch * P.H_I * 128) + off),
+                       tc::sdesc_kmajor_sw128(tc::smem_u32(sB + (gc & 1) * bytesB + ch * NW * 128) + off),
                        idesc, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(aempty(s));
@@ -282,57 +317,107 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue: one entry per thread ----
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    UnitWalk wk;
+    UnitWalk<G> wk;
     wk.start(P, prefix, u0);
-    int last_q = -1;
-    int64_t nv = 0;
-    float* out = nullptr;
-    const float* wq = nullptr;
-    float wr[HREG > 0 ? HREG : 1];
-    for (int i = 0; i < nunits; ++i, wk.next()) {
-      const int q = wk.q;
-      if (q != last_q) {
-        nv = dec_nvis(P, q);
-        out = P.scores + (int64_t)q * P.ld_scores;
-        wq = P.w + (int64_t)q * P.H_I;
+    if constexpr (G > 1) {
+      constexpr int GH = G / 2;             // queries of the group this warp reduces
+      const int j0 = (warp - 2) / 4 * GH;   // warps 2-5: the first half, 6-9: the second
+      int last_q = -1;
+      int64_t nv[GH];
+      for (int i = 0; i < nunits; ++i, wk.next()) {
+        const int g = wk.q;
+        if (g != last_q) {
+#pragma unroll
+          for (int j = 0; j < GH; ++j) {
+            const int q = g * G + j0 + j;
+            nv[j] = q < P.Q ? dec_nvis(P, q) : 0;
+          }
+          last_q = g;
+        }
+        const int a = i % NACC;
+        if (!tc::mbar_wait_warp(accfull(a), (i / NACC) & 1, P.err)) break;
+        tc::tc_fence_after();
+        float sc[GH];
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj) {
+          const int j = j0 + jj;
+          sc[jj] = 0.f;
+          const int q = g * G + j;
+          if (q >= P.Q) continue;  // same for the whole warp
+          // H_I = 64 here; the same four chains over the heads as for G = 1
+          const float* wq = P.w + (int64_t)q * 64;
+          float v[64];
+          tc::tmem_ld64(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * NW + j * 64), v);
+          float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int h = 0; h < 64; h += 4) {
+            const float4 w4 = __ldg(reinterpret_cast<const float4*>(wq + h));
+            acc4[0] = fmaf(w4.x, fmaxf(v[h], 0.f), acc4[0]);
+            acc4[1] = fmaf(w4.y, fmaxf(v[h + 1], 0.f), acc4[1]);
+            acc4[2] = fmaf(w4.z, fmaxf(v[h + 2], 0.f), acc4[2]);
+            acc4[3] = fmaf(w4.w, fmaxf(v[h + 3], 0.f), acc4[3]);
+          }
+          sc[jj] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(accempty(a));
+        const int64_t sidx = wk.t * kTileM + row;
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj)
+          if (sidx < nv[jj]) P.scores[(int64_t)(g * G + j0 + jj) * P.ld_scores + sidx] = sc[jj];
+      }
+    } else {
+      int last_q = -1;
+      int64_t nv = 0;
+      float* out = nullptr;
+      const float* wq = nullptr;
+      float wr[HREG > 0 ? HREG : 1];
+      for (int i = 0; i < nunits; ++i, wk.next()) {
+        const int q = wk.q;
+        if (q != last_q) {
+          nv = dec_nvis(P, q);
+          out = P.scores + (int64_t)q * P.ld_scores;
+          wq = P.w + (int64_t)q * P.H_I;
+          if (HREG > 0) {
+#pragma unroll
+            for (int h = 0; h < HREG; h += 4) {
+              const float4 t4 = __ldg(reinterpret_cast<const float4*>(wq + h));
+              wr[h] = t4.x;
+              wr[h + 1] = t4.y;
+              wr[h + 2] = t4.z;
+              wr[h + 3] = t4.w;
+            }
+          }
+          last_q = q;
+        }
+        const int a = i % NACC;
+        if (!tc::mbar_wait_warp(accfull(a), (i / NACC) & 1, P.err)) break;
+        tc::tc_fence_after();
+        float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains over the heads
         if (HREG > 0) {
 #pragma unroll
-          for (int h = 0; h < HREG; h += 4) {
-            const float4 t4 = __ldg(reinterpret_cast<const float4*>(wq + h));
-            wr[h] = t4.x;
-            wr[h + 1] = t4.y;
-            wr[h + 2] = t4.z;
-            wr[h + 3] = t4.w;
+          for (int h0 = 0; h0 < (HREG > 0 ? HREG : 16); h0 += 32) {
+            float v[32];
+            tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * HREG + h0), v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc4[j & 3] = fmaf(wr[h0 + j], fmaxf(v[j], 0.f), acc4[j & 3]);
+          }
+        } else {
+          for (int h0 = 0; h0 < P.H_I; h0 += 16) {
+            float v[16];
+            tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * P.H_I + h0), v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc4[j & 3] = fmaf(__ldg(wq + h0 + j), fmaxf(v[j], 0.f), acc4[j & 3]);
           }
         }
-        last_q = q;
+        const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(accempty(a));
+        const int64_t sidx = wk.t * kTileM + row;
+        if (sidx < nv) out[sidx] = acc;
       }
-      const int a = i % kDecAcc;
-      if (!tc::mbar_wait_warp(accfull(a), (i / kDecAcc) & 1, P.err)) break;
-      tc::tc_fence_after();
-      float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains over the heads
-      if (HREG > 0) {
-#pragma unroll
-        for (int h0 = 0; h0 < (HREG > 0 ? HREG : 16); h0 += 32) {
-          float v[32];
-          tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * HREG + h0), v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc4[j & 3] = fmaf(wr[h0 + j], fmaxf(v[j], 0.f), acc4[j & 3]);
-        }
-      } else {
-        for (int h0 = 0; h0 < P.H_I; h0 += 16) {
-          float v[16];
-          tc::tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * P.H_I + h0), v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) acc4[j & 3] = fmaf(__ldg(wq + h0 + j), fmaxf(v[j], 0.f), acc4[j & 3]);
-        }
-      }
-      const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(accempty(a));
-      const int64_t sidx = wk.t * kTileM + row;
-      if (sidx < nv) out[sidx] = acc;
     }
   }
   tc::tc_fence_before();
@@ -353,11 +438,15 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
                                    const int64_t* n_entries, int Q, int H_I, int c_I,
                                    float* scores, int64_t ld_scores, cudaStream_t s) {
   if (Q == 0 || ldK == 0 || nseq == 0) return cudaSuccess;
+  // w rows are read as float4 by the register and grouped paths
+  const bool w16 = (reinterpret_cast<uintptr_t>(w) & 15) == 0;
+  // one sequence and many queries (prefill): groups of 4 queries share each key tile
+  const int G = (nseq == 1 && H_I == 64 && c_I <= 128 && w16 && Q >= 64) ? 4 : 1;
   CUtensorMap tmK, tmQ;
   if (!encode_tmap_2d_bf16(&tmK, KI, (uint64_t)c_I, (uint64_t)nseq * ldK, (uint64_t)c_I * 2, 64,
                            kTileM) ||
       !encode_tmap_2d_bf16(&tmQ, qI, (uint64_t)c_I, (uint64_t)Q * H_I, (uint64_t)c_I * 2, 64,
-                           (uint32_t)H_I))
+                           (uint32_t)(G * H_I)))
     return cudaErrorInvalidValue;
   DecParams P{};
   P.Q = Q;
@@ -378,25 +467,29 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  P.interleave = Q >= 4 * nsm ? 1 : 0;
+  P.NG = (Q + G - 1) / G;
+  P.interleave = P.NG >= 4 * nsm ? 1 : 0;
+  const int nacc = G == 1 ? kDecAcc : kGrpAcc;
   uint32_t cols = 32;
-  while (cols < (uint32_t)(kDecAcc * H_I)) cols <<= 1;
+  while (cols < (uint32_t)(nacc * G * H_I)) cols <<= 1;
+  if (cols > 512) return cudaErrorInvalidValue;
   P.tmem_cols = cols;
   const int KCH = c_I / 64;
-  const size_t prefix_ints = P.interleave ? 2 : (size_t)Q + 3;
-  const size_t fixed = 1024 + 2 * (size_t)KCH * H_I * 128 + 128 * 4 + prefix_ints * 4 + 256;
+  const size_t prefix_ints = P.interleave ? 2 : (size_t)P.NG + 3;
+  const size_t fixed = 1024 + 2 * (size_t)KCH * G * H_I * 128 + prefix_ints * 4 + 256;
   const size_t per_stage = (size_t)KCH * kChunkBytesA;
-  const int stages = (int)std::min<size_t>(6, (220 * 1024 - fixed) / per_stage);
-  if (stages < 2) return cudaErrorInvalidValue;
+  // the grouped kernel takes all of shared memory (two 64 KB query groups + 3 stages)
+  const size_t cap = G > 1 ? 227 * 1024 : 220 * 1024;
+  if (fixed + 2 * per_stage > cap) return cudaErrorInvalidValue;
+  const int stages = (int)std::min<size_t>(6, (cap - fixed) / per_stage);
   P.stages = stages;
   const size_t smem = fixed + stages * per_stage;
-  // w rows are read as float4 in the register path: 16-byte aligned rows
-  const bool wreg = H_I == 64 && (reinterpret_cast<uintptr_t>(w) & 15) == 0;
-  auto kern = wreg ? index_decode_kernel<64> : index_decode_kernel<0>;
+  auto kern = G > 1 ? index_decode_kernel<0, 4>
+                    : (H_I == 64 && w16 ? index_decode_kernel<64, 1> : index_decode_kernel<0, 1>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   count_launches();
-  kern<<<nsm, kThreads, smem, s>>>(tmK, tmQ, P);
+  kern<<<nsm, G > 1 ? GroupCfg<4>::threads : GroupCfg<1>::threads, smem, s>>>(tmK, tmQ, P);
   return cudaGetLastError();
 }
 

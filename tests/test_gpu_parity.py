@@ -242,6 +242,24 @@ def test_index_topk_grouped_queries(orc, HI, cI):
         assert max_abs(sc[q, :nv], ref["scores"][q, :nv]) <= 2.0 ** -14 * ref["amag"][q] + 1e-6
 
 
+@pytest.mark.parametrize("Q", [257, 2501])
+def test_index_topk_single_sequence_groups_bit_exact(orc, Q):
+    """One sequence, many queries (the prefill shape): queries are scored in
+    groups of four that share each entry tile. Unsorted positions give the
+    members of a group different visible counts (some none); Q is not a
+    multiple of four; 257 queries split the units into contiguous ranges,
+    2501 deal whole groups to CTAs in turn. Integer inputs make every score
+    exact, so the selected sets must equal the oracle's."""
+    N, k = 300, 64
+    qI, w, KI, seq, pos, ne = _index_inputs(Q, 64, 128, 1, N, "bf16", integer=True, seed=21)
+    rg = np.random.default_rng(22)
+    pos[:] = rg.integers(0, 4 * N + 16, Q)
+    pos[:6] = [0, 3, 4, 4 * N + 3, 2, 1]
+    idx = _run_index(qI, w, KI, seq, pos, ne, k, "bf16").cpu().numpy()
+    want = orc.index_topk(qI, w, KI, seq, pos, ne, m=4, k=k)["idx"]
+    np.testing.assert_array_equal(idx, want)
+
+
 @pytest.mark.parametrize("k", [1024, 300])
 def test_index_topk_many_entries_bit_exact(orc, k):
     """More visible entries than one selection block holds: chunk top-k
