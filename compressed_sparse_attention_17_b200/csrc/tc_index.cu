@@ -51,12 +51,17 @@ template <int G>
 struct GroupCfg {
   static constexpr int acc = G == 1 ? kDecAcc : kGrpAcc;
   static constexpr int epi_warps = G == 1 ? 4 : 8;
+  // qI slots: two for single queries (the next query loads while the current
+  // one is multiplied); one 64 KB slot for groups, which leaves room for a
+  // fourth key stage (the next group's qI is first pulled into L2)
+  static constexpr int qslots = G == 1 ? 2 : 1;
   static constexpr int threads = 64 + 32 * epi_warps;
 };
 
 struct DecParams {
   int Q, H_I, c_I, nseq, stages;
   int NG;  // query groups of G consecutive queries
+  const void* qI;
   int64_t ldK;
   int m, vis_offset;
   const int32_t* seq_of_q;
@@ -165,12 +170,15 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
   const int NW = G * P.H_I;  // MMA N: the group's (query, head) rows
   const int bytesA = KCH * kChunkBytesA;
   const int bytesB = KCH * NW * 128;
+  constexpr int QS = GroupCfg<G>::qslots;
   uint8_t* sA = smem;
   uint8_t* sB = sA + S * bytesA;
-  int* prefix = reinterpret_cast<int*>(sB + 2 * bytesB);
+  // groups: the head weights of two groups (double-buffered, bulk-copied)
+  float* wsm = reinterpret_cast<float*>(sB + QS * bytesB);
+  int* prefix = reinterpret_cast<int*>(wsm + (G > 1 ? 2 * NW : 0));
   uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + (P.interleave ? 2 : ((P.NG + 2 + 1) & ~1)));
-  // bars: Afull[S], Aempty[S], Bfull[2], Bempty[2], accfull[NACC], accempty[NACC]
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4 + 2 * NACC);
+  // bars: Afull[S], Aempty[S], Bfull[2], Bempty[2], accfull[NACC], accempty[NACC], Wfull[2], Wempty[2]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4 + 2 * NACC + 4);
   constexpr int kThreads = GroupCfg<G>::threads;
   constexpr int kEpi = GroupCfg<G>::epi_warps;
   __shared__ int scan_tmp[kThreads / 32];
@@ -226,6 +234,8 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
   auto bempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 2 + s]); };
   auto accfull = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + s]); };
   auto accempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + NACC + s]); };
+  auto wfull = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + 2 * NACC + s]); };
+  auto wempty = [&](int s) { return tc::smem_u32(&bars[2 * S + 4 + 2 * NACC + 2 + s]); };
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(afull(s), 1);
@@ -238,6 +248,10 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
     for (int s = 0; s < NACC; ++s) {
       tc::mbar_init(accfull(s), 1);
       tc::mbar_init(accempty(s), kEpi);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(wfull(s), 1);
+      tc::mbar_init(wempty(s), kEpi);
     }
     tc::fence_barrier_init();
     tc::prefetch_tmap(&tmK);
@@ -257,18 +271,21 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
       UnitWalk<G> wk;
       wk.start(P, prefix, u0);
       int last_q = -1, gc = -1;
+      // qI of a new query (group) into its slot once the slot's previous
+      // occupant has left the MMA
+      auto load_q = [&](int q) {
+        ++gc;
+        const int bs = gc % QS;
+        if (gc >= QS && !tc::mbar_wait(bempty(bs), ((gc / QS) - 1) & 1, P.err)) return false;
+        tc::mbar_arrive_expect_tx(bfull(bs), (uint32_t)bytesB);
+        for (int ch = 0; ch < KCH; ++ch)
+          tc::tma_load_2d(tc::smem_u32(sB + bs * bytesB + ch * NW * 128), &tmQ, ch * 64, q * NW, bfull(bs));
+        return true;
+      };
       for (int i = 0; i < nunits; ++i, wk.next()) {
         const int q = wk.q;
-        if (q != last_q) {
-          ++gc;
-          const int bs = gc & 1;
-          if (gc >= 2 && !tc::mbar_wait(bempty(bs), ((gc >> 1) - 1) & 1, P.err)) break;
-          tc::mbar_arrive_expect_tx(bfull(bs), (uint32_t)bytesB);
-          for (int ch = 0; ch < KCH; ++ch)
-            tc::tma_load_2d(tc::smem_u32(sB + bs * bytesB + ch * NW * 128), &tmQ, ch * 64, q * NW,
-                            bfull(bs));
-          last_q = q;
-        }
+        const bool newq = q != last_q;
+        if (G == 1 && newq && !load_q(q)) break;
         const int s = i % S;
         if (i >= S && !tc::mbar_wait(aempty(s), ((i / S) - 1) & 1, P.err)) break;
         tc::mbar_arrive_expect_tx(afull(s), (uint32_t)bytesA);
@@ -278,6 +295,26 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
         for (int ch = 0; ch < KCH; ++ch)
           tc::tma_load_2d_hint(tc::smem_u32(sA + s * bytesA + ch * kChunkBytesA), &tmK, ch * 64, y,
                                afull(s), pol);
+        if (G > 1 && newq) {
+          // the key tile goes first: it needs no qI slot and lands while the
+          // previous group drains from the single slot
+          if (!load_q(q)) break;
+          const int ws = gc & 1;
+          if (gc >= 2 && !tc::mbar_wait(wempty(ws), ((gc >> 1) - 1) & 1, P.err)) break;
+          const uint32_t wbytes = (uint32_t)(min(G, P.Q - q * G) * P.H_I * 4);
+          tc::mbar_arrive_expect_tx(wfull(ws), wbytes);
+          tc::bulk_copy_g2s(tc::smem_u32(wsm + ws * NW), P.w + (int64_t)q * NW, wbytes, wfull(ws));
+          // the next group's qI into L2, so that its load at the next change
+          // is an L2 hit
+          const int qn = P.interleave ? q + (int)gridDim.x : q + 1;
+          if (qn < P.NG) {
+            const int64_t r0 = (int64_t)qn * NW;
+            const int64_t r1 = min((int64_t)(qn + 1) * NW, (int64_t)P.Q * P.H_I);
+            tc::prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(P.qI) + r0 * P.c_I * 2,
+                                 (uint32_t)((r1 - r0) * P.c_I * 2));
+          }
+        }
+        last_q = q;
       }
     }
     __syncwarp();
@@ -291,9 +328,9 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
       for (int i = 0; i < nunits; ++i, wk.next()) {
         const int q = wk.q;
         if (q != last_q) {
-          if (gc >= 0) tc::mma_commit(bempty(gc & 1));  // previous query's qI slot is free
+          if (gc >= 0) tc::mma_commit(bempty(gc % QS));  // previous query's qI slot is free
           ++gc;
-          if (!tc::mbar_wait(bfull(gc & 1), (gc >> 1) & 1, P.err)) break;
+          if (!tc::mbar_wait(bfull(gc % QS), (gc / QS) & 1, P.err)) break;
           last_q = q;
         }
         const int s = i % S, a = i % NACC;
@@ -305,7 +342,7 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
           const int ch = kk >> 2;
           const uint32_t off = (uint32_t)(kk & 3) * 32;
           tc::mma_bf16(d, tc::sdesc_kmajor_sw128(tc::smem_u32(sA + s * bytesA + ch * kChunkBytesA) + off),
-                       tc::sdesc_kmajor_sw128(tc::smem_u32(sB + (gc & 1) * bytesB + ch * NW * 128) + off),
+                       tc::sdesc_kmajor_sw128(tc::smem_u32(sB + (gc % QS) * bytesB + ch * NW * 128) + off),
                        idesc, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(aempty(s));
@@ -322,11 +359,17 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
     if constexpr (G > 1) {
       constexpr int GH = G / 2;             // queries of the group this warp reduces
       const int j0 = (warp - 2) / 4 * GH;   // warps 2-5: the first half, 6-9: the second
-      int last_q = -1;
+      int last_q = -1, gce = -1;
       int64_t nv[GH];
+      const float* wg = wsm;
       for (int i = 0; i < nunits; ++i, wk.next()) {
         const int g = wk.q;
         if (g != last_q) {
+          // the previous group's weights are no longer read by this warp
+          if (gce >= 0 && lane == 0) tc::mbar_arrive(wempty(gce & 1));
+          ++gce;
+          if (!tc::mbar_wait_warp(wfull(gce & 1), (gce >> 1) & 1, P.err)) break;
+          wg = wsm + (gce & 1) * NW;
 #pragma unroll
           for (int j = 0; j < GH; ++j) {
             const int q = g * G + j0 + j;
@@ -345,13 +388,13 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
           const int q = g * G + j;
           if (q >= P.Q) continue;  // same for the whole warp
           // H_I = 64 here; the same four chains over the heads as for G = 1
-          const float* wq = P.w + (int64_t)q * 64;
+          const float* wq = wg + j * 64;  // shared memory: one broadcast read per four heads
           float v[64];
           tc::tmem_ld64(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * NW + j * 64), v);
           float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int h = 0; h < 64; h += 4) {
-            const float4 w4 = __ldg(reinterpret_cast<const float4*>(wq + h));
+            const float4 w4 = *reinterpret_cast<const float4*>(wq + h);
             acc4[0] = fmaf(w4.x, fmaxf(v[h], 0.f), acc4[0]);
             acc4[1] = fmaf(w4.y, fmaxf(v[h + 1], 0.f), acc4[1]);
             acc4[2] = fmaf(w4.z, fmaxf(v[h + 2], 0.f), acc4[2]);
@@ -468,6 +511,7 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   P.NG = (Q + G - 1) / G;
+  P.qI = qI;
   P.interleave = P.NG >= 4 * nsm ? 1 : 0;
   const int nacc = G == 1 ? kDecAcc : kGrpAcc;
   uint32_t cols = 32;
@@ -476,9 +520,11 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
   P.tmem_cols = cols;
   const int KCH = c_I / 64;
   const size_t prefix_ints = P.interleave ? 2 : (size_t)P.NG + 3;
-  const size_t fixed = 1024 + 2 * (size_t)KCH * G * H_I * 128 + prefix_ints * 4 + 256;
+  const int qslots = G > 1 ? GroupCfg<4>::qslots : GroupCfg<1>::qslots;
+  const size_t fixed = 1024 + (size_t)qslots * KCH * G * H_I * 128 +
+                       (G > 1 ? 2 * (size_t)G * H_I * 4 : 0) + prefix_ints * 4 + 256;
   const size_t per_stage = (size_t)KCH * kChunkBytesA;
-  // the grouped kernel takes all of shared memory (two 64 KB query groups + 3 stages)
+  // the grouped kernel takes all of shared memory (one 64 KB query group + 4 stages)
   const size_t cap = G > 1 ? 227 * 1024 : 220 * 1024;
   if (fixed + 2 * per_stage > cap) return cudaErrorInvalidValue;
   const int stages = (int)std::min<size_t>(6, (cap - fixed) / per_stage);
