@@ -247,6 +247,27 @@ class Prefill:
         torch.cuda.synchronize(device)
         log(f"[prefill] setup {time.time() - t0:.1f}s: T={T}")
 
+    def time_scores(self, reps, warmup, flush):
+        """Device ms of the indexer alone (csa_index_scores on the step's
+        index keys), L2 flushed before each launch, outside the events."""
+        t = self.t
+        sc = torch.empty(self.w.T, self.KI.shape[0], device=self.dev)
+        call = lambda: csa.index_scores(t["qI"], t["w"], self.KI[None], self.seq, self.pos,
+                                        self.ne, self.g, out=sc)
+        for _ in range(warmup):
+            flush_l2(flush)
+            call()
+        ev = []
+        for _ in range(reps):
+            flush_l2(flush)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            ev.append((a, b))
+        torch.cuda.synchronize(self.dev)
+        return [a.elapsed_time(b) for a, b in ev]
+
     def index_flops(self):
         """Algorithmic FLOPs of the prefill indexer: 2 H_I c_I per visible
         (query, entry) pair, entry s visible to token t when s < (t + 1) / m."""
@@ -268,6 +289,7 @@ class Prefill:
                        out=self.idx)
         if ev:
             ev[1].record()
+        self.KI = KI
         csa.attend(t["q"], t["sink"], E[None], self.idx, win[None], self.seq, self.pos, self.ne,
                    self.g, out=self.O)
 
@@ -534,15 +556,20 @@ def main():
                    "unit": "tokens/s", "ms_per_step": pms_max,
                    "config": {"workload": pw.name, "T": pw.T, "d": pw.d, "top_k": pw.k}}
         if csa_pre:
-            # tensor roofline of the indexer: the whole csa_index_topk call
-            # (score launch + top-k launch) against the indexer's FLOPs alone
+            # tensor roofline of the indexer: the score kernel alone
+            # (csa_index_scores, timed in its own loop), and the step's whole
+            # csa_index_topk call (score launch + top-k launch) beside it
+            sms = max_over_ranks(statistics.mean(pre.time_scores(max(5, args.steps // 2), 3, flush)))
             ims_max = max_over_ranks(statistics.mean(ims))
             fl = pre.index_flops()
-            ach = fl / (ims_max / 1e3) / 1e12
+            ach = fl / (sms / 1e3) / 1e12
             prefill["indexer_roofline"] = {
                 "bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
-                "frac": ach / tflops, "kernel": "csa_index_topk (prefill, indexer + top-k launches)",
-                "kernel_ms": ims_max, "algorithmic_flop": fl,
+                "frac": ach / tflops,
+                "kernel": f"csa_index_scores (prefill, {pw.T} queries)",
+                "kernel_ms": sms, "algorithmic_flop": fl,
+                "index_topk_call_ms": ims_max,
+                "index_topk_call_frac": fl / (ims_max / 1e3) / 1e12 / tflops,
                 "peak_source": f"{peak_kind} dense BF16 GEMM (burst)"}
         del pre
 

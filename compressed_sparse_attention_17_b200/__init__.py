@@ -67,6 +67,8 @@ _SIGS = {
     "csa_index_topk_workspace_size": ([_I32, _I64, _I32], _SZ),
     "csa_index_topk": ([_GP, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _I32, _I32, _I32,
                         _P, _P, _P, _SZ, _P], _I32),
+    "csa_index_scores": ([_GP, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _I32, _I32, _P,
+                          _I64, _P], _I32),
     "csa_index_topk_noalloc": ([_GP, _I32, _P, _P, _P, _I64, _I32, _P, _P, _P, _I32, _I32, _I32,
                                 _I32, _P, _P, _P], _I32),
     "csa_attend_workspace_size": ([_I32, _I32, _I32, _I32, _I32], _SZ),
@@ -221,6 +223,19 @@ def index_topk(qI, w, KI, seq_of_q, pos, n_entries, k, g: Geom, want_scores=Fals
           KI.shape[0], _ptr(seq_of_q), _ptr(pos), _ptr(n_entries), Q, HI, cI, k, _ptr(idx), _ptr(scores),
           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(qI))
     return (idx, scores) if want_scores else idx
+
+
+def index_scores(qI, w, KI, seq_of_q, pos, n_entries, g: Geom, out=None):
+    """Indexer scores I [Q, ldK] (FP32) for the visible entries of each query;
+    the other slots of a new buffer hold NaN."""
+    _check(qI, w, KI, seq_of_q, pos, n_entries)
+    Q, HI, cI = qI.shape
+    ldK = KI.shape[1]
+    sc = out if out is not None else torch.full((Q, ldK), float("nan"), device=qI.device)
+    _call("csa_index_scores", ctypes.byref(g), _dt(qI), _ptr(qI), _ptr(w), _ptr(KI), ldK,
+          KI.shape[0], _ptr(seq_of_q), _ptr(pos), _ptr(n_entries), Q, HI, cI, _ptr(sc),
+          sc.shape[1], _stream(qI))
+    return sc
 
 
 def attend(q, sink, E, idx, win, seq_of_q, pos, n_entries, g: Geom, q_gain=None, out=None,

@@ -226,6 +226,28 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
                                       idx_out, scores_dbg, ldK, cand, s));
 }
 
+csa_status csa_index_scores(const csa_geom* g, csa_dtype dtype, const void* qI, const float* w,
+                            const void* KI, int64_t ldK, int nseq, const int32_t* seq_of_q,
+                            const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
+                            int c_I, float* scores, int64_t ld_scores, csa_stream_t stream) {
+  if (!geom_ok(g) || !io_dtype_ok(dtype)) return CSA_ERR_INVALID_ARG;
+  if (Q < 0 || H_I < 1 || H_I > 128 || c_I < 16 || (c_I % 16) != 0 || c_I > 256) return CSA_ERR_INVALID_ARG;
+  if (ldK < 0 || nseq < 0 || ld_scores < ldK) return CSA_ERR_INVALID_ARG;
+  if (Q == 0 || ldK == 0 || nseq == 0) return CSA_OK;
+  if (!qI || !w || !KI || !seq_of_q || !pos || !n_entries || !scores) return CSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {qI, w, KI, seq_of_q, pos, n_entries, scores};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return CSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = csa::index_tc_supported(dtype, H_I, c_I)
+                      ? csa::launch_index_scores_tc(*g, qI, w, KI, ldK, nseq, seq_of_q, pos,
+                                                    n_entries, Q, H_I, c_I, scores, ld_scores, s)
+                      : csa::launch_index_scores_simt(*g, dtype, qI, w, KI, ldK, nseq, seq_of_q,
+                                                      pos, n_entries, Q, H_I, c_I, scores,
+                                                      ld_scores, s);
+  return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}
+
 size_t csa_attend_workspace_size(int Q, int H_q, int c, int k, int n_win) {
   (void)Q, (void)H_q, (void)c, (void)k, (void)n_win;
   return 0;

@@ -11,6 +11,15 @@
 namespace csa {
 
 // ---------------------------------------------------------------- errors
+// Programmatic dependent launch: a kernel launched with launch_pdl()
+// (internal.h) is scheduled as soon as the previous kernel's blocks have all
+// exited, and runs its setup while that kernel's writes drain. pdl_wait()
+// returns once that kernel has completed and its writes are visible (a no-op
+// for ordinary launches). No kernel signals its successor early: measured on
+// the decode step, successors that were scheduled while a persistent kernel
+// still ran slowed it down.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Bounded device-side waits that give up record a status code in the
 // library's device error word (defined in api.cu, passed to kernels as a
 // pointer); csa_sync_status() reads and clears it.

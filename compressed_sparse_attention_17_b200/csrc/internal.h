@@ -16,6 +16,27 @@ int* device_error_ptr();
 // Counts one kernel launch (csa_kernel_launches()).
 void count_launches(int n = 1);
 
+// Launch with programmatic dependent launch allowed: the kernel may be
+// scheduled while the previous kernel of the stream finishes. Every kernel
+// launched this way calls pdl_wait() (common.cuh) before its first access to
+// global memory, so it still observes everything that kernel wrote and
+// writes nothing that kernel still reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---- SIMT kernels (simt.cu): every dtype, every shape the ABI accepts ----
 cudaError_t launch_rmsnorm_rope(const csa_geom& g, int in_dt, int out_dt, const void* x,
                                 int64_t rows, const int64_t* pos, int64_t pos0, int64_t pos_step,

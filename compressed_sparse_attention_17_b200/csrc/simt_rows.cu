@@ -29,6 +29,7 @@ __global__ void rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int
                                     int64_t pos0, int64_t pos_step, const float* __restrict__ gain,
                                     void* __restrict__ out, const int64_t* __restrict__ out_row,
                                     int out_dt, int do_norm, int do_rope) {
+  pdl_wait();
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -375,6 +376,7 @@ __global__ void __launch_bounds__(kPoolThreads) decode_pool_kernel(
     const float* __restrict__ gain, const float* __restrict__ state, int out_dt,
     void* __restrict__ E, int64_t ldE) {
   __shared__ float red[kPoolThreads / 32];
+  pdl_wait();
   const int b = blockIdx.x;
   const int c = g.c, m = g.m;
   const int64_t p = pos[b];
@@ -437,14 +439,12 @@ cudaError_t launch_rmsnorm_rope(const csa_geom& g, int in_dt, int out_dt, const 
   count_launches();
   dim3 block(256), grid((unsigned)((rows + 7) / 8));
   if (in_dt == CSA_F32)
-    rmsnorm_rope_kernel<float><<<grid, block, 0, s>>>(
-        reinterpret_cast<const float*>(x), rows, g.c, g.rope_dims, g.rope_base, g.eps, pos, pos0,
-        pos_step, gain, out, out_row, out_dt, 1, 1);
-  else
-    rmsnorm_rope_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        reinterpret_cast<const __nv_bfloat16*>(x), rows, g.c, g.rope_dims, g.rope_base, g.eps,
-        pos, pos0, pos_step, gain, out, out_row, out_dt, 1, 1);
-  return cudaGetLastError();
+    return launch_pdl(rmsnorm_rope_kernel<float>, grid, block, 0, s,
+                      reinterpret_cast<const float*>(x), rows, g.c, g.rope_dims, g.rope_base,
+                      g.eps, pos, pos0, pos_step, gain, out, out_row, out_dt, 1, 1);
+  return launch_pdl(rmsnorm_rope_kernel<__nv_bfloat16>, grid, block, 0, s,
+                    reinterpret_cast<const __nv_bfloat16*>(x), rows, g.c, g.rope_dims,
+                    g.rope_base, g.eps, pos, pos0, pos_step, gain, out, out_row, out_dt, 1, 1);
 }
 
 cudaError_t launch_quantize_mixed(int in_dt, const void* x, int64_t rows, void* out,
@@ -510,8 +510,8 @@ cudaError_t launch_decode_pool(const csa_geom& g, const int64_t* pos, int B, con
                                int64_t ldE, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   count_launches();
-  decode_pool_kernel<<<B, kPoolThreads, 0, s>>>(g, pos, bias, gain, state, out_dt, E, ldE);
-  return cudaGetLastError();
+  return launch_pdl(decode_pool_kernel, dim3(B), dim3(kPoolThreads), 0, s, g, pos, bias, gain,
+                    state, out_dt, E, ldE);
 }
 
 }  // namespace csa

@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
   float* inv_den = reinterpret_cast<float*>(sm + kOffInv);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();  // the previous kernel's writes (the selected entries) are visible from here on
   const int qi = blockIdx.x;
   const int b = P.seq_of_q[qi];
   const int64_t p = P.pos[qi];
@@ -524,8 +525,7 @@ cudaError_t launch_attend_tc(const csa_geom& g, int kv_dt, const void* q, const 
                                        (int)smem);
   if (e != cudaSuccess) return e;
   count_launches();
-  attend_tc_kernel<<<(unsigned)Q, kThreads, smem, s>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(attend_tc_kernel, dim3((unsigned)Q), dim3(kThreads), smem, s, P);
 }
 
 }  // namespace csa

@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return tc::smem_u32(&bars[i]); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();  // the previous kernel's writes (the selected entries) are visible from here on
   const int C = P.csize;
   const int rank = (int)(blockIdx.x % (unsigned)C);
   const int qi = (int)(blockIdx.x / (unsigned)C);
@@ -740,13 +741,15 @@ cudaError_t launch_attend_cluster(const csa_geom& g, int kv_dt, const void* q, c
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)P.csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   count_launches();
   return cudaLaunchKernelEx(&cfg, attend_cluster_kernel, tq, P);
 }

@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(GroupCfg<G>::threads, 1)
   constexpr int kThreads = GroupCfg<G>::threads;
   constexpr int kEpi = GroupCfg<G>::epi_warps;
   __shared__ int scan_tmp[kThreads / 32];
+  pdl_wait();  // the previous kernel's writes are visible from here on
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -535,8 +536,8 @@ cudaError_t launch_index_scores_tc(const csa_geom& g, const void* qI, const floa
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   count_launches();
-  kern<<<nsm, G > 1 ? GroupCfg<4>::threads : GroupCfg<1>::threads, smem, s>>>(tmK, tmQ, P);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(nsm), dim3(G > 1 ? GroupCfg<4>::threads : GroupCfg<1>::threads),
+                    smem, s, tmK, tmQ, P);
 }
 
 }  // namespace csa

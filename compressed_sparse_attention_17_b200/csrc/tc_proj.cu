@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();               // inputs of the previous kernel visible from here on
 
   if (warp == 0 && lane == 0) {
     // ---- TMA producer ----
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(256) decode_reduce_kernel(const float* __restr
                                                             int m, int overlap,
                                                             const int64_t* __restrict__ pos,
                                                             float* __restrict__ state) {
+  pdl_wait();
   const int ncols = nW * c;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (int64_t)B * ncols) return;
@@ -272,8 +274,8 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap* tmW, const Params&
                                        kSmem);
   if (e != cudaSuccess) return e;
   count_launches();
-  proj_tc_kernel<<<grid, kThreads, kSmem, s>>>(tmA, tmW[0], tmW[1], tmW[2], tmW[3], P);
-  return cudaGetLastError();
+  return launch_pdl(proj_tc_kernel, grid, dim3(kThreads), kSmem, s, tmA, tmW[0], tmW[1], tmW[2],
+                    tmW[3], P);
 }
 
 int decode_ksplit(int ntiles, int mtiles, int total_chunks, int* chunks_per_split) {
@@ -360,9 +362,8 @@ cudaError_t launch_decode_proj_tc(const csa_geom& g, const void* h, const int64_
   if (e != cudaSuccess) return e;
   const int64_t n = (int64_t)B * nW * g.c;
   count_launches();
-  decode_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, ksplit, B, nW, g.c, g.m,
-                                                                   g.overlap, pos, state);
-  return cudaGetLastError();
+  return launch_pdl(decode_reduce_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
+                    (const float*)part, ksplit, B, nW, g.c, g.m, g.overlap, pos, state);
 }
 
 }  // namespace csa

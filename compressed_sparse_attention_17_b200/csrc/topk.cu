@@ -205,6 +205,7 @@ __device__ __forceinline__ int chunk_len(const Params& P, int64_t nv, int c) {
 template <int NT, int KPT, bool CAND>
 __global__ void __launch_bounds__(NT, CAND ? 1 : 1024 / NT) topk_cluster_kernel(Params P) {
   __shared__ Smem<NT> S;
+  pdl_wait();  // the scores of the previous kernel are visible from here on
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int C = P.csize, kpt = P.kpt, k = P.k;
   const int rank = (int)(blockIdx.x % (unsigned)C);
@@ -548,13 +549,15 @@ cudaError_t launch_one(const Params& P, int64_t nseg, cudaStream_t s) {
   cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)P.csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   count_launches();
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<NT, KPT, CAND>, P);
 }

@@ -228,6 +228,19 @@ csa_status csa_index_topk(const csa_geom* g, csa_dtype dtype, const void* qI, co
                           void* workspace, size_t ws_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------
+ * csa_index_scores - the lightning indexer's scores alone, without the
+ * selection (the same equation, arguments and visibility as csa_index_topk).
+ *   scores    [Q, ld_scores] FP32, ld_scores >= ldK: I[q, s] for
+ *             s < n_vis(q); slots s >= n_vis(q) are left untouched.
+ * The scores are bit-identical to the ones csa_index_topk selects from.
+ * No workspace. Errors as for csa_index_topk.
+ * --------------------------------------------------------------------- */
+csa_status csa_index_scores(const csa_geom* g, csa_dtype dtype, const void* qI, const float* w,
+                            const void* KI, int64_t ldK, int nseq, const int32_t* seq_of_q,
+                            const int64_t* pos, const int64_t* n_entries, int Q, int H_I,
+                            int c_I, float* scores, int64_t ld_scores, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------
  * csa_index_topk_noalloc - csa_index_topk without a caller workspace.
  * (An interface addition of this library; the pages have no counterpart.)
  * For callers that cannot allocate device memory around the call - code

@@ -242,6 +242,23 @@ def test_index_topk_grouped_queries(orc, HI, cI):
         assert max_abs(sc[q, :nv], ref["scores"][q, :nv]) <= 2.0 ** -14 * ref["amag"][q] + 1e-6
 
 
+@pytest.mark.parametrize("dt,HI,cI,Q,nseq", [("bf16", 64, 128, 300, 1), ("bf16", 64, 128, 40, 3),
+                                           ("f32", 4, 32, 40, 3)])
+def test_index_scores_integer_inputs_bit_exact(orc, dt, HI, cI, Q, nseq):
+    """csa_index_scores alone: integer inputs make every score exact, so the
+    visible slots equal the oracle's scores; grouped queries (one sequence),
+    single queries and the CUDA-core path."""
+    qI, w, KI, seq, pos, ne = _index_inputs(Q, HI, cI, nseq, 700, dt, integer=True, seed=31)
+    g = csa.geom(m=4, vis_offset=1)
+    sc = csa.index_scores(dev(qI, dt), dev(w, "f32"), dev(KI, dt), dev_i(seq, torch.int32),
+                          dev_i(pos), dev_i(ne), g).cpu().numpy()
+    ref = orc.index_topk(qI, w, KI, seq, pos, ne, m=4, k=8, want_scores=True)["scores"]
+    for q in range(Q):
+        nv = orc.visible_entries(pos[q], 4, 1, ne[seq[q]])
+        np.testing.assert_array_equal(sc[q, :nv], ref[q, :nv])
+        assert np.isnan(sc[q, nv:]).all()
+
+
 @pytest.mark.parametrize("Q", [257, 2501])
 def test_index_topk_single_sequence_groups_bit_exact(orc, Q):
     """One sequence, many queries (the prefill shape): queries are scored in
