@@ -172,7 +172,7 @@ class Decode:
         log(f"[decode] setup {time.time() - t0:.1f}s: B={B} entries={N} "
             f"{'mixed FP8' if mixed else 'BF16'} cache")
 
-    def step(self, inp, ev=None):
+    def step(self, inp, ev=None, O=None):
         W = self.W
         csa.compress_decode(inp["h"], inp["pos"], W["W_aKV"], W["W_aZ"], self.bias, self.state,
                             self.E, self.g, W_bKV=W["W_bKV"], W_bZ=W["W_bZ"])
@@ -187,7 +187,7 @@ class Decode:
         if ev is not None:
             ev[1].record()
         csa.attend(inp["q"], self.sink, self.E, self.idx, self.ring, self.seq, inp["pos"],
-                   self.ne, self.g, out=self.O)
+                   self.ne, self.g, out=self.O if O is None else O)
 
     def capture(self):
         """Record one decode step (all of its library launches) as a CUDA
@@ -202,16 +202,62 @@ class Decode:
     def step_graph(self, ev=None):
         self.graph.replay()
 
-    def step_e2e(self):
-        """Same step through the public API from pinned host buffers:
-        inputs copied host->device and the output copied back."""
-        for n, t in self.host.items():
-            self.inp[n].copy_(t, non_blocking=True)
+    def setup_pipeline(self):
+        """A second set of step inputs and outputs (and, with graphs, a second
+        graph on them), so that one step's copies overlap another's kernels."""
+        second = {n: t.clone() for n, t in self.inp.items()}
+        self.inp2 = [self.inp, second]
+        self.O2 = [self.O, torch.empty_like(self.O)]
+        self.host_O2 = [self.host_O, torch.empty_like(self.host_O).pin_memory()]
+        self.graphs = None
         if getattr(self, "graph", None) is not None:
-            self.graph.replay()
-        else:
-            self.step(self.inp)
-        self.host_O.copy_(self.O, non_blocking=True)
+            self.step(second, O=self.O2[1])
+            torch.cuda.synchronize(self.dev)
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                self.step(second, O=self.O2[1])
+            self.graphs = [self.graph, g2]
+        self.s_h2d = torch.cuda.Stream(self.dev)
+        self.s_d2h = torch.cuda.Stream(self.dev)
+        torch.cuda.synchronize(self.dev)
+
+    def run_pipelined(self, nsteps):
+        """nsteps decode steps through the public API from pinned host
+        buffers, the way a serving loop runs them: step i's inputs are copied
+        host->device on one stream while step i-1's kernels run on the current
+        stream, and each step's output is copied back on a third stream. The
+        two buffer sets alternate; events keep a set from being overwritten
+        while a step still reads it. Returns events around the whole run
+        (first input copy to last output copy)."""
+        sc = torch.cuda.current_stream(self.dev)
+        sh, sd = self.s_h2d, self.s_d2h
+        ev = lambda: torch.cuda.Event()
+        h_done, c_done, d_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(sh)
+        for i in range(nsteps):
+            b = i & 1
+            with torch.cuda.stream(sh):
+                if i >= 2:
+                    sh.wait_event(c_done[b])  # step i-2 no longer reads these inputs
+                for n, t in self.host.items():
+                    self.inp2[b][n].copy_(t, non_blocking=True)
+                h_done[b].record(sh)
+            sc.wait_event(h_done[b])
+            if i >= 2:
+                sc.wait_event(d_done[b])  # step i-2's output has been copied out
+            if self.graphs is not None:
+                self.graphs[b].replay()
+            else:
+                self.step(self.inp2[b], O=self.O2[b])
+            c_done[b].record(sc)
+            with torch.cuda.stream(sd):
+                sd.wait_event(c_done[b])
+                self.host_O2[b].copy_(self.O2[b], non_blocking=True)
+                d_done[b].record(sd)
+        end.record(sd)
+        return start, end
 
     @property
     def h2d_bytes(self):
@@ -441,7 +487,9 @@ def main():
     config = {"workload": w.name, "launch": "host" if args.no_graph else "cuda_graph", "batch": w.B, "context": w.L, "entries_per_seq": w.n_entries,
               "m": w.m, "top_k": w.k, "window": w.n_win, "query_heads": w.H_q, "head_dim": w.c,
               "indexer_heads": w.H_I, "indexer_dim": w.c_I, "parallelism": f"dp{args.gpus}",
-              "l2": "flushed (256 MiB write) before every timed step"}
+              "l2": "flushed (256 MiB write) before every timed step",
+              "e2e": "pinned host inputs copied in and the output copied back every step; "
+                     "steps pipelined over three streams; no flush (each step streams > L2)"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -499,23 +547,18 @@ def main():
     ms_max = max_over_ranks(ms)
     value = whole_job_rate(w.B, args.gpus, ms_max)
 
-    # end to end through the public API from pinned host memory
+    # end to end through the public API from pinned host memory: steps
+    # pipelined over three streams (copies of one step overlap the kernels of
+    # the previous one); no L2 flush between steps, each of which streams more
+    # than 300 MB of cache through L2
     e2e_ms = None
     if not args.no_e2e:
-        for _ in range(args.warmup):
-            flush_l2(flush)
-            dec.step_e2e()
+        dec.setup_pipeline()
+        dec.run_pipelined(args.warmup)
         torch.cuda.synchronize(device)
-        e2e = []
-        for _ in range(args.steps):
-            flush_l2(flush)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            dec.step_e2e()
-            b.record()
-            e2e.append((a, b))
+        a, b = dec.run_pipelined(args.steps)
         torch.cuda.synchronize(device)
-        e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e))
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps)
     h2d_bytes, d2h_bytes = dec.h2d_bytes, dec.d2h_bytes
 
     # roofline of the dominant kernel (the indexer)
@@ -548,7 +591,8 @@ def main():
         pw = synth.WORKLOADS[args.prefill_workload]()
         pre = (Prefill if pw.kind == "csa_prefill" else HcaPrefill)(pw, device)
         csa_pre = pw.kind == "csa_prefill"
-        pms, ims = time_steps(lambda ev: pre.step(ev), max(3, args.steps // 4), 3, device, flush,
+        pms, ims = time_steps((lambda ev: pre.step(ev)) if csa_pre else (lambda ev: pre.step()),
+                              max(3, args.steps // 4), 3, device, flush,
                               extra_events=2 if csa_pre else 0)
         pms_max = max_over_ranks(statistics.mean(pms))
         prefill = {"metric": ("CSA" if pw.kind == "csa_prefill" else "HCA") + " prefill tokens/s",

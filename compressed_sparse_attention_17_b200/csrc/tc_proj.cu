@@ -278,6 +278,10 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap* tmW, const Params&
                     tmW[3], P);
 }
 
+// Split-K factor of a decode projection: about enough splits that the N
+// tiles times the splits fill the SMs once, at most 16 (the partials are
+// summed by decode_reduce_kernel; 64 splits of the 512-wide index-key
+// projection, which has two N tiles, made the decode step slower).
 int decode_ksplit(int ntiles, int mtiles, int total_chunks, int* chunks_per_split) {
   const int target = min(16, max(1, 148 / max(1, ntiles * mtiles)));
   const int cps = max(1, (total_chunks + target - 1) / target);
