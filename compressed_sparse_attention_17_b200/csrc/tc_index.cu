@@ -4,11 +4,12 @@
 // ("Evidence Ledger", CSA Eqs 13-17; "DeepSeek-V4" study 03, index-score
 // formula).
 //
-// A tile of 128 compressed entries against one query: the entries are the
-// MMA's M dimension (one TMEM lane each), the query's heads its N dimension,
-// the key width its K dimension. TMA brings both operands into shared memory
-// in the 128-byte-swizzled K-major layout; one thread issues tcgen05.mma into
-// a TMEM accumulator; four epilogue warps read their lanes back and apply the
+// A tile of 128 compressed entries against one query, or against a group of
+// four consecutive queries of one sequence: the entries are the MMA's M
+// dimension (one TMEM lane each), the (query, head) rows its N dimension, the
+// key width its K dimension. TMA brings both operands into shared memory in
+// the 128-byte-swizzled K-major layout; one thread issues tcgen05.mma into a
+// TMEM accumulator; the epilogue warps read their lanes back and apply the
 // ReLU, the head weights and the head sum in registers, so each thread owns
 // one entry and no cross-thread reduction is needed.
 //
