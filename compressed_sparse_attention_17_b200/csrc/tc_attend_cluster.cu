@@ -462,27 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pw = warp - 4;
     const int row_bytes_e = (int)row_bytes(P.kv_dt, kDim);
     const bool mixed_kv = P.kv_dt == CSA_FP8_MIXED;
-    // Every row of this CTA's tiles is requested into L2 first: the DRAM
-    // reads of all tiles then overlap, and each tile's gather below waits
-    // only for L2.
-    {
-      const int64_t s_end = min((t0 + T) * (int64_t)kTile, nslots);
-      for (int64_t slot = t0 * kTile + (threadIdx.x - 128); slot < s_end; slot += 128) {
-        const uint8_t* row = nullptr;
-        uint32_t nb = (uint32_t)row_bytes_e;
-        if (slot < nsel) {
-          const int64_t e = P.dense ? slot : (int64_t)list[slot];
-          row = reinterpret_cast<const uint8_t*>(P.E) + ((int64_t)b * ldE + e) * row_bytes_e;
-        } else {
-          const int64_t j = w0 + (slot - nsel);
-          const int64_t wr = P.win_ring ? (j % P.n_win) : j;
-          nb = 2u * kDim;
-          if (wr < P.ldW) row = reinterpret_cast<const uint8_t*>(P.win + ((int64_t)b * P.ldW + wr) * kDim);
-        }
-        if (row != nullptr && ((reinterpret_cast<uintptr_t>(row) | nb) & 15u) == 0)
-          tc::prefetch_l2_bulk(row, nb);
-      }
-    }
     for (int t = 0; t < T; ++t) {
       const int buf = t & 1;
       if (t >= 2 && !tc::mbar_wait_warp(bar(kEmpty0 + buf), (uint32_t)((t >> 1) - 1) & 1u, P.err))
