@@ -326,10 +326,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
     // ---- S^T = K Qhat^T ----
     if (warp == 8 && lane == 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(128, kHeads);
+      const uint64_t dk = tc::sdesc_kmajor_sw128(sK), dq = tc::sdesc_kmajor_sw128(sQ);
+#pragma unroll 4
       for (int kk = 0; kk < kDim / 16; ++kk) {
         const uint32_t ch = kk >> 2, off = (uint32_t)(kk & 3) * 32;
-        tc::mma_bf16(tmem + kColS, tc::sdesc_kmajor_sw128(sK + ch * 16384 + off),
-                     tc::sdesc_kmajor_sw128(sQ + ch * 8192 + off), idesc, kk > 0);
+        tc::mma_bf16(tmem + kColS, tc::sdesc_add(dk, ch * 16384 + off), tc::sdesc_add(dq, ch * 8192 + off),
+                     idesc, kk > 0 ? 1u : 0u);
       }
       tc::mma_commit(s_bar);
     }
@@ -404,12 +406,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(Params P) {
     if (warp == 8 && lane == 0) {
       if (!flags[0]) {
         const uint32_t idesc = tc::idesc_bf16_f32_major(128, kHeads, 1, 1);
+        const uint64_t da = tc::sdesc_mnmajor_sw128(sK, 16384, 1024);
+        const uint64_t db = tc::sdesc_mnmajor_sw128(sP, 8192, 1024);
+        const uint32_t acc0 = t > t_begin ? 1u : 0u;
+#pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t ad = tc::sdesc_mnmajor_sw128(sK + (2 * blk) * 16384 + kk * 2048, 16384, 1024);
-            const uint64_t bd = tc::sdesc_mnmajor_sw128(sP + kk * 2048, 8192, 1024);
-            tc::mma_bf16(tmem + kColO + blk * kHeads, ad, bd, idesc, (t > t_begin || kk > 0) ? 1u : 0u);
-          }
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            tc::mma_bf16(tmem + kColO + blk * kHeads, tc::sdesc_add(da, (2 * blk) * 16384 + kk * 2048),
+                         tc::sdesc_add(db, kk * 2048), idesc, kk > 0 ? 1u : acc0);
         }
       }
       tc::mma_commit(o_bar);

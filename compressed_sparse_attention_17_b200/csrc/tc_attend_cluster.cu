@@ -524,10 +524,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = ns & 1;
         tc::tc_fence_after();
         const uint32_t kb = sK + buf * kTileBytes;
+        const uint64_t dq = tc::sdesc_kmajor_sw128(sQ), dk = tc::sdesc_kmajor_sw128(kb);
+        const uint32_t ds = tmem + kColS + buf * 64;
+#pragma unroll 4
         for (int kk = 0; kk < kDim / 16; ++kk) {
-          const uint32_t ch = kk >> 2, off = (uint32_t)(kk & 3) * 32;
-          tc::mma_bf16(tmem + kColS + buf * 64, tc::sdesc_kmajor_sw128(sQ + ch * 8192 + off),
-                       tc::sdesc_kmajor_sw128(kb + ch * 8192 + off), id_s, kk > 0);
+          const uint32_t o = (uint32_t)((kk >> 2) * 8192 + (kk & 3) * 32);
+          tc::mma_bf16(ds, tc::sdesc_add(dq, o), tc::sdesc_add(dk, o), id_s, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(bar(kSFull0 + buf));
         ++ns;
@@ -537,12 +539,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = npv & 1;
         tc::tc_fence_after();
         const uint32_t kb = sK + buf * kTileBytes;
+        const uint64_t da = tc::sdesc_mnmajor_sw128(kb, 8192, 1024);
+        const uint64_t db = tc::sdesc_kmajor_sw128(sP + buf * 8192);
+        const uint32_t acc0 = npv > 0 ? 1u : 0u;
+#pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t ad = tc::sdesc_mnmajor_sw128(kb + (2 * blk) * 8192 + kk * 2048, 8192, 1024);
-            const uint64_t bd = tc::sdesc_kmajor_sw128(sP + buf * 8192 + kk * 32);
-            tc::mma_bf16(tmem + kColO + blk * kHeads, ad, bd, id_pv, (npv > 0 || kk > 0) ? 1u : 0u);
-          }
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            tc::mma_bf16(tmem + kColO + blk * kHeads, tc::sdesc_add(da, (2 * blk) * 8192 + kk * 2048),
+                         tc::sdesc_add(db, kk * 32), id_pv, kk > 0 ? 1u : acc0);
         }
         tc::mma_commit(bar(kEmpty0 + buf));
         tc::mma_commit(bar(kODone));

@@ -292,6 +292,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, int a_
   return idesc_bf16_f32(M, N) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 }
 
+// Descriptor d with its start address advanced by `bytes` (a multiple of
+// 16). The address sits in the low 14 bits as address / 16 and shared-memory
+// addresses stay below 256 KB, so the sum never carries out of the field.
+// Issue loops build each operand's descriptor once and advance it with
+// constant offsets: building it per instruction costs the issuing thread
+// about as long as a small MMA takes to run.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
+}
+
 // Shared-memory descriptor of an MN-major operand with 128-byte swizzling:
 // 64 BF16 along M/N contiguous per 128-byte row, rows = consecutive K,
 // 8-row groups `sbo` bytes apart, 64-element M/N blocks `lbo` bytes apart.
