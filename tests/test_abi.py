@@ -89,6 +89,18 @@ def test_index_topk_argument_checks(lib):
     assert lib.csa_index_topk(*args(16, 64, 128, None, 0)) == 1         # no workspace
 
 
+def test_index_scores_argument_checks(lib):
+    g = csa.geom()
+    args = lambda HI, cI, sc, ld, w=OK: (ctypes.byref(g), 1, OK, w, OK, 100, 1, OK, OK, OK, 4, HI,
+                                         cI, sc, ld, None)
+    assert lib.csa_index_scores(*args(64, 100, OK, 100)) == 1      # c_I % 16
+    assert lib.csa_index_scores(*args(300, 128, OK, 100)) == 1     # H_I > 128
+    assert lib.csa_index_scores(*args(64, 128, OK, 99)) == 1       # ld_scores < ldK
+    assert lib.csa_index_scores(*args(64, 128, None, 100)) == 1    # no output
+    assert lib.csa_index_scores(*args(64, 128, BAD, 100)) == 1     # misaligned output
+    assert lib.csa_index_scores(*args(64, 128, OK, 100, w=None)) == 1  # no weights
+
+
 def test_compress_argument_checks(lib):
     g = csa.geom()
     # CSA without the b-series weights
