@@ -188,6 +188,8 @@ class Decode:
             ev[1].record()
         csa.attend(inp["q"], self.sink, self.E, self.idx, self.ring, self.seq, inp["pos"],
                    self.ne, self.g, out=self.O if O is None else O)
+        if ev is not None and len(ev) > 2:
+            ev[2].record()
 
     def capture(self):
         """Record one decode step (all of its library launches) as a CUDA
@@ -266,6 +268,13 @@ class Decode:
     @property
     def d2h_bytes(self):
         return self.O.numel() * self.O.element_size()
+
+    def attend_bytes(self):
+        """Algorithmic bytes of one attention launch: the selected entry rows
+        and the window rows of every query, its queries in and outputs out."""
+        w = self.w
+        row = csa.MIXED_ROW_BYTES if w.kv_mixed else 2 * w.c
+        return w.B * (w.k * row + w.n_win * 2 * w.c) + 2 * w.B * w.H_q * w.c * 2
 
     def index_bytes(self):
         """Algorithmic bytes of one indexer launch: every visible index key
@@ -537,6 +546,21 @@ def main():
     # the indexer launch alone, for the roofline (events on the launching stream)
     _, idx_ms = time_steps(lambda ev: dec.step(dec.inp, ev), max(5, args.steps // 2), args.warmup,
                            device, flush, extra_events=2)
+    # the indexer and the attention together (csa_index_topk then csa_attend,
+    # events before the first and after the second), in a loop of their own
+    ia_ms = None
+    try:
+        evs = []
+        for i in range(args.warmup + max(5, args.steps // 2)):
+            flush_l2(flush)
+            e3 = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            dec.step(dec.inp, e3)
+            if i >= args.warmup:
+                evs.append(e3)
+        torch.cuda.synchronize(device)
+        ia_ms = statistics.mean(e3[0].elapsed_time(e3[2]) for e3 in evs)
+    except Exception as ex:  # optional figure: reported as absent rather than failing the run
+        log(f"[decode] indexer + attention timing unavailable: {ex}")
     if not args.no_graph:
         dec.capture()
     barrier()
@@ -577,6 +601,14 @@ def main():
             traffic = rec.get("dram_bytes_per_launch") if same else None
         except (ValueError, OSError):
             traffic = None
+    index_attention = None
+    if ia_ms is not None:
+        ia_ms = max_over_ranks(ia_ms)
+        ia_bytes = idx_bytes + dec.attend_bytes()
+        ia_ach = ia_bytes / (ia_ms / 1e3) / 1e9
+        index_attention = {"bound": "hbm", "achieved": ia_ach, "peak": hbm, "unit": "GB/s",
+                           "frac": ia_ach / hbm, "ms": ia_ms, "algorithmic_bytes": ia_bytes,
+                           "calls": "csa_index_topk + csa_attend (decode step)"}
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic,
                 "kernel": f"csa_index_topk (decode, all {w.B} queries)",
@@ -639,6 +671,7 @@ def main():
                         "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
                 "gpu_launches": per_step_launches * args.steps,
                 "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+                "decode_index_attention": index_attention,
                 "prefill": prefill}
         print(json.dumps(line), flush=True)
     if torch.distributed.is_initialized():

@@ -36,3 +36,15 @@ def test_decode_indexer_bytes_are_the_tensors_read():
     selected = w.B * w.k * 4                        # the int32 indices written
     assert dec.index_bytes() == keys + queries + weights + selected
     assert keys == 32 * 32768 * 128 * 2
+
+
+def test_decode_attention_bytes_are_the_rows_read():
+    w = synth.csa_decode_bf16()
+    dec = bench.Decode.__new__(bench.Decode)
+    dec.w = w
+    # 32 queries x (1024 selected + 128 window) rows of 512 BF16, queries in and outputs out
+    assert dec.attend_bytes() == 32 * 1152 * 1024 + 2 * (32 * 64 * 512 * 2)
+    mixed = synth.csa_decode_long_mixed()
+    dec.w = mixed
+    # selected rows in the 592-byte mixed format, window rows in BF16
+    assert dec.attend_bytes() == 4 * (1024 * 592 + 128 * 1024) + 2 * (4 * 64 * 512 * 2)
